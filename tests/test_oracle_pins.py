@@ -1,0 +1,352 @@
+"""Pins of the CPU oracle to facts it does not compute itself.
+
+Each `check_*` function below tests the oracle module passed to it against a
+hand derivation, a closed form, a brute-force loop, a library routine, or an
+invariant of the mathematics.  The plain tests run them on the real oracle; the
+mutation tests at the end plant a plausible mistake in a copy of one oracle
+function (on the CPU, in this process) and require that some check fails.
+"""
+
+import json
+import math
+import os
+import types
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import oracle.convrot_oracle as real_oracle
+import workloads
+
+pytestmark = pytest.mark.filterwarnings("ignore::RuntimeWarning")
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+H4_HALF = np.array([[1, 1, 1, 1], [1, -1, 1, -1], [1, 1, -1, -1], [1, -1, -1, 1]], np.float64) / 2
+
+
+def _golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+# ---------------------------------------------------------------------------
+# checks (each takes the oracle module)
+# ---------------------------------------------------------------------------
+
+def check_worked_example(o):
+    """Hand-derived G = 4 example (tests/golden/hadamard4_worked_example.json)."""
+    g = _golden("hadamard4_worked_example.json")
+    x, W, b = (np.array(g[k], np.float64) for k in ("x", "W", "bias"))
+    np.testing.assert_array_equal(o.block_rotate(x, H4_HALF), np.array(g["x_rot"]))
+    np.testing.assert_array_equal(o.block_rotate(W, H4_HALF), np.array(g["W_rot"]))
+    xq, s_tok = o.rotate_quant_act(x, H4_HALF)
+    np.testing.assert_array_equal(xq, np.array(g["xq"]))
+    assert s_tok[0] == np.float32(5 / 127)
+    Wq, s_w = o.quantize_weight(W, H4_HALF)
+    np.testing.assert_array_equal(Wq, np.array(g["Wq"]))
+    assert s_w == np.float32(5 / 127)
+    acc = o.int8_gemm_acc(xq, Wq)
+    np.testing.assert_array_equal(acc, np.array(g["acc"]))
+    np.testing.assert_array_equal(o.epilogue(acc, s_tok, s_w, b), np.array(g["y"]))
+    np.testing.assert_array_equal(o.dequant_derotate(Wq, s_w, H4_HALF), np.array(g["W_hat"]))
+    np.testing.assert_array_equal(o.linear_dense(x, W, b), np.array(g["y_dense"]))
+
+
+def check_block_rotate_bruteforce(o):
+    """Against explicit loops over the definition (x B_R)[r, b*G+j] = sum_i x[r, b*G+i] R[i, j]."""
+    rng = np.random.default_rng(7)
+    for G in (4, 16):
+        K = 3 * G
+        A = rng.standard_normal((3, K))
+        R = rng.standard_normal((G, G))
+        out = o.block_rotate(A, R)
+        ref = np.zeros_like(A)
+        for r in range(3):
+            for b in range(K // G):
+                for j in range(G):
+                    ref[r, b * G + j] = sum(A[r, b * G + i] * R[i, j] for i in range(G))
+        np.testing.assert_allclose(out, ref, rtol=1e-13, atol=1e-13)
+
+
+def check_block_rotate_direction(o):
+    """A one-hot input e_{b*G+i} rotates to row i of R inside block b, zeros elsewhere."""
+    R = workloads.qr_rotation(16, seed=11).astype(np.float64)
+    G, K = 16, 48
+    for b, i in ((0, 0), (1, 5), (2, 15)):
+        e = np.zeros((1, K))
+        e[0, b * G + i] = 1.0
+        out = o.block_rotate(e, R)[0]
+        expect = np.zeros(K)
+        expect[b * G:(b + 1) * G] = R[i]
+        np.testing.assert_array_equal(out, expect)
+
+
+def check_rotation_identity(o):
+    """x W^T = (x B_R)(W B_R)^T for an orthogonal R (float64, rel 1e-12)."""
+    rng = np.random.default_rng(3)
+    q, r = np.linalg.qr(rng.standard_normal((64, 64)))
+    R = q * np.sign(np.diag(r))
+    x = rng.standard_normal((5, 256))
+    W = rng.standard_normal((7, 256))
+    lhs = x @ W.T
+    rhs = o.block_rotate(x, R) @ o.block_rotate(W, R).T
+    assert np.max(np.abs(lhs - rhs)) <= 1e-12 * np.max(np.abs(lhs))
+
+
+def check_round_trip(o):
+    """Derotation undoes rotation: decode of an unquantized rotated weight is W."""
+    R = workloads.qr_rotation(64, seed=5).astype(np.float64)
+    R, _ = np.linalg.qr(R)  # re-orthogonalise in float64 so the inverse is exact to rounding
+    W = np.random.default_rng(1).standard_normal((6, 128))
+    back = o.block_rotate(o.block_rotate(W, R), R.T)
+    np.testing.assert_allclose(back, W, rtol=0, atol=1e-13)
+
+
+def check_bf16_round(o):
+    """bf16 rounding: equals torch's float32 -> bfloat16 conversion on float32
+    inputs, and rounds float64 inputs once (no detour through float32)."""
+    rng = np.random.default_rng(0)
+    v = np.concatenate([
+        rng.standard_normal(20000) * 10.0 ** rng.integers(-6, 6, 20000),
+        np.array([0.0, -0.0, 1.0, -1.0, 1 + 2 ** -8, 1 + 3 * 2 ** -8, -(1 + 2 ** -8), 3.0e38 / 4]),
+    ]).astype(np.float32)
+    ref = torch.from_numpy(v).to(torch.bfloat16).float().numpy().astype(np.float64)
+    np.testing.assert_array_equal(o.bf16_round(v.astype(np.float64)), ref)
+    # ties to even: 1 + 2^-8 lies half way between 1 and 1 + 2^-7 -> 1
+    assert o.bf16_round(1 + 2 ** -8) == 1.0
+    # 1 + 3*2^-8 lies half way between 1 + 2^-7 and 1 + 2^-6 -> the even one, 1 + 2^-6
+    assert o.bf16_round(1 + 3 * 2 ** -8) == 1 + 2 ** -6
+    # just above the tie: float32 would first round it onto the tie (then to even = 1),
+    # a single rounding from float64 goes up.
+    assert o.bf16_round(1 + 2 ** -8 + 2 ** -40) == 1 + 2 ** -7
+    assert o.bf16_round(-(1 + 2 ** -8 + 2 ** -40)) == -(1 + 2 ** -7)
+
+
+def check_quantize_symmetric(o):
+    """round half to even, clamp to +-127, zero scale -> zero codes."""
+    s = np.float32(1.0)
+    v = np.array([2.5, 3.5, -2.5, -3.5, 0.49, 126.5, 127.4, 200.0, -300.0])
+    np.testing.assert_array_equal(o.quantize_symmetric(v, s), [2, 4, -2, -4, 0, 126, 127, 127, -127])
+    np.testing.assert_array_equal(o.quantize_symmetric(np.array([1.0, -3.0]), np.float32(0.0)), [0, 0])
+
+
+def check_act_quant_properties(o):
+    """Per token: s_tok = max|x_rot| / 127 (float32), the largest entry maps to
+    +-127, codes lie in [-127, 127], and |x_rot - q s_tok| <= s_tok / 2."""
+    lin = workloads.Linear("t", 37, 512, 8, G=64)
+    x = workloads.make_layer_inputs(lin, 9).x
+    R = workloads.sylvester_rotation(64)
+    xq, s_tok = o.rotate_quant_act(x, R)
+    x_rot = o.block_rotate(x, R)
+    a = np.max(np.abs(x_rot), axis=1)
+    np.testing.assert_array_equal(s_tok, (a / 127).astype(np.float32))
+    assert xq.dtype == np.int8 and xq.min() >= -127 and xq.max() <= 127
+    np.testing.assert_array_equal(np.max(np.abs(xq.astype(np.int32)), axis=1), 127)
+    err = np.abs(x_rot - xq.astype(np.float64) * s_tok[:, None].astype(np.float64))
+    assert np.all(err <= s_tok[:, None] * (0.5 + 1e-5))
+
+
+def check_zero_token(o):
+    """An all-zero token: s_tok = 0, codes 0, output row = bf16(bias)."""
+    R = workloads.sylvester_rotation(16)
+    x = np.zeros((2, 32))
+    x[1, 3] = 1.0
+    W = np.random.default_rng(2).standard_normal((4, 32)) * 0.02
+    bias = np.array([0.25, -0.5, 1.0, 0.0])
+    Wq, s_w = o.quantize_weight(W, R)
+    y, xq, s_tok, acc = o.linear_int8(x, Wq, s_w, R, bias)
+    assert s_tok[0] == 0 and not xq[0].any() and not acc[0].any()
+    np.testing.assert_array_equal(y[0], bias)
+    assert np.any(y[1] != bias)
+
+
+def check_gemm_bruteforce(o):
+    """int8 GEMM against Python-integer triple loops on small random codes."""
+    rng = np.random.default_rng(4)
+    a = rng.integers(-127, 128, (5, 40), dtype=np.int64).astype(np.int8)
+    b = rng.integers(-127, 128, (6, 40), dtype=np.int64).astype(np.int8)
+    acc = o.int8_gemm_acc(a, b)
+    assert acc.dtype == np.int32
+    for m in range(5):
+        for n in range(6):
+            assert int(acc[m, n]) == sum(int(a[m, k]) * int(b[n, k]) for k in range(40))
+
+
+def check_gemm_extremes(o):
+    """The largest accumulator of the workloads (K = 15360) is exact."""
+    K = 15360
+    a = np.full((2, K), 127, np.int8)
+    a[1] = -127
+    b = np.full((1, K), 127, np.int8)
+    acc = o.int8_gemm_acc(a, b)
+    assert acc[0, 0] == 127 * 127 * K and acc[1, 0] == -127 * 127 * K
+    # alternating signs cancel exactly
+    c = np.tile(np.array([127, -127], np.int8), K // 2)[None, :]
+    assert o.int8_gemm_acc(c, b)[0, 0] == 0
+
+
+def check_epilogue_closed_forms(o):
+    acc = np.array([[0, 1, -3, 1 << 20]], np.int32)
+    bias = np.array([0.5, -0.25, 2.0, 0.0])
+    np.testing.assert_array_equal(o.epilogue(acc * 0, np.float32([0.1]), np.float32(3.0), bias), [bias])
+    np.testing.assert_array_equal(o.epilogue(acc, np.float32([1.0]), np.float32(1.0)), [[0, 1, -3, 2.0 ** 20]])
+    # 257 is not a bf16 (needs 9 bits) and is half way between 256 and 258 -> 256 (even)
+    np.testing.assert_array_equal(o.epilogue(np.array([[257]]), np.float32([1.0]), np.float32(1.0)), [[256.0]])
+
+
+def check_weight_decode_accuracy(o):
+    """Decode of a rotated int8 weight against the bf16 weight.
+
+    PR #194 "QA Instructions" measures decoded corr 0.99978-1.0 on real weights
+    and PR #10185 cosine 0.99996; the SenseNova page puts the per-layer weight
+    reconstruction error well below 2 %.  The synthetic weights' 1 % outlier
+    columns (x10) set a larger per-tensor scale than real weights do, so the
+    pin is the pages' lower end, cosine >= 0.9998, and rel-L2 < 2 %.  Without
+    the derotation the cosine collapses (the pages' negative control: 0.054-0.065
+    and 0.06 on real weights)."""
+    lin = workloads.Linear("t", 1, 1024, 256)
+    W = workloads.make_layer_inputs(lin, 0).W
+    for R in (workloads.sylvester_rotation(256), workloads.qr_rotation(256)):
+        Wq, s_w = o.quantize_weight(W, R)
+        W_hat = o.dequant_derotate(Wq, s_w, R)
+        assert o.cosine(W_hat, W) >= 0.9998
+        assert o.rel_l2(W_hat, W) < 0.02
+        assert abs(o.cosine(np.float64(s_w) * Wq.astype(np.float64), W)) < 0.1
+
+
+def check_layer_accuracy(o):
+    """int8 layer against the unquantized float64 layer: cosine >= 0.999."""
+    lin = workloads.WORKLOADS["single_1024"][0]
+    for rot in ("sylvester", "qr"):
+        inp = workloads.make_layer_inputs(lin, 0, rotation=rot)
+        Wq, s_w = o.quantize_weight(inp.W, inp.R)
+        y, *_ = o.linear_int8(inp.x, Wq, s_w, inp.R, inp.bias)
+        assert o.cosine(y, o.linear_dense(inp.x, inp.W, inp.bias)) >= 0.999
+
+
+def check_rotation_helps_outliers(o):
+    """Int8 Compute page, "Layer / Why": without the rotation one outlier channel
+    sets the scale of the whole token.  Per-token quantization error of the
+    activations is clearly lower with R = H than with R = I."""
+    x = workloads.make_activation(64, 1024, 1000, 4, 2000)
+    errs = {}
+    for name, R in (("H", workloads.sylvester_rotation(256)), ("I", np.eye(256))):
+        xq, s_tok = o.rotate_quant_act(x, R)
+        x_rot = o.block_rotate(x, R)
+        errs[name] = o.rel_l2(xq.astype(np.float64) * s_tok[:, None], x_rot)
+    assert errs["H"] < 0.25 * errs["I"]
+
+
+CHECKS = [
+    check_worked_example, check_block_rotate_bruteforce, check_block_rotate_direction,
+    check_rotation_identity, check_round_trip, check_bf16_round, check_quantize_symmetric,
+    check_act_quant_properties, check_zero_token, check_gemm_bruteforce, check_gemm_extremes,
+    check_epilogue_closed_forms, check_weight_decode_accuracy, check_layer_accuracy,
+    check_rotation_helps_outliers,
+]
+
+
+@pytest.mark.parametrize("check", CHECKS, ids=lambda c: c.__name__)
+def test_oracle_pin(check):
+    check(real_oracle)
+
+
+def test_rotations_orthogonal():
+    """The rotation blocks the workloads draw are orthogonal: Sylvester exactly,
+    the float32-stored QR matrix to float32 rounding."""
+    for G in workloads.GROUP_SIZES:
+        R = workloads.sylvester_rotation(G).astype(np.float64)
+        np.testing.assert_array_equal(R @ R.T, np.eye(G))
+        assert set(np.unique(np.abs(R))) == {2.0 ** (-math.log2(G) / 2)}
+        Q = workloads.qr_rotation(G).astype(np.float64)
+        assert np.max(np.abs(Q @ Q.T - np.eye(G))) < 1e-6
+
+
+# ---------------------------------------------------------------------------
+# planted mistakes: each must make at least one check fail
+# ---------------------------------------------------------------------------
+
+def _mutant(**overrides):
+    m = types.ModuleType("oracle_mutant")
+    m.__dict__.update({k: v for k, v in vars(real_oracle).items() if not k.startswith("__")})
+    m.__dict__.update(overrides)
+    # functions resolve globals through their own module; rebind them to the mutant
+    for name, fn in list(m.__dict__.items()):
+        if isinstance(fn, types.FunctionType) and name not in overrides:
+            m.__dict__[name] = types.FunctionType(fn.__code__, m.__dict__, name, fn.__defaults__)
+    return m
+
+
+def _bug_skip_derotation(Wq, s_w, R):
+    return real_oracle.bf16_round(np.float64(np.float32(s_w)) * np.asarray(Wq, np.float64))
+
+
+def _bug_transposed_rotation(A, R):
+    A = real_oracle.as_f64(A)
+    R = real_oracle.as_f64(R).T
+    G = R.shape[0]
+    return (A.reshape(A.shape[0], -1, G) @ R).reshape(A.shape)
+
+
+def _bug_drop_bias(acc, s_tok, s_w, bias=None):
+    return real_oracle.epilogue(acc, s_tok, s_w, None)
+
+
+def _bug_group_scale(x, R):
+    # codes taken with a per-group scale while the row scale is reported
+    x_rot = real_oracle.block_rotate(x, R)
+    G = np.asarray(R).shape[0]
+    M, K = x_rot.shape
+    g = x_rot.reshape(M, K // G, G)
+    sg = (np.max(np.abs(g), axis=2, keepdims=True) / 127).astype(np.float32)
+    q = real_oracle.quantize_symmetric(g, sg).reshape(M, K)
+    return q, (np.max(np.abs(x_rot), axis=1) / 127).astype(np.float32)
+
+
+def _bug_gemm_k_off_by_one(xq, Wq):
+    return real_oracle.int8_gemm_acc(np.asarray(xq)[:, :-1], np.asarray(Wq)[:, :-1])
+
+
+def _bug_truncating_round(v, scale):
+    v32 = np.asarray(v, np.float64).astype(np.float32)
+    s32 = np.broadcast_to(np.asarray(scale, np.float32), v32.shape)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        q = np.trunc(v32 / s32)
+    return np.clip(np.where(s32 == 0, 0, q), -127, 127).astype(np.int8)
+
+
+def _bug_bf16_via_fp32(v):
+    f = np.asarray(v, np.float64).astype(np.float32)
+    return torch.from_numpy(np.atleast_1d(f)).to(torch.bfloat16).double().numpy().reshape(np.shape(f))
+
+
+def _bug_scale_255(W, R):
+    W_rot = real_oracle.block_rotate(W, R)
+    s_w = np.float32(np.max(np.abs(W_rot)) / 255)
+    return real_oracle.quantize_symmetric(W_rot, s_w), s_w
+
+
+MUTANTS = {
+    "skip_derotation": dict(dequant_derotate=_bug_skip_derotation),
+    "transposed_rotation": dict(block_rotate=_bug_transposed_rotation),
+    "drop_bias": dict(epilogue=_bug_drop_bias),
+    "per_group_act_scale": dict(rotate_quant_act=_bug_group_scale),
+    "gemm_drops_last_k": dict(int8_gemm_acc=_bug_gemm_k_off_by_one),
+    "truncating_round": dict(quantize_symmetric=_bug_truncating_round),
+    "bf16_double_rounding": dict(bf16_round=_bug_bf16_via_fp32),
+    "weight_scale_255": dict(quantize_weight=_bug_scale_255),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_planted_mistake_is_caught(name):
+    m = _mutant(**MUTANTS[name])
+    failed = []
+    for check in CHECKS:
+        try:
+            check(m)
+        except (AssertionError, ValueError, OverflowError):
+            failed.append(check.__name__)
+    assert failed, f"planted mistake {name!r} passed every check"
