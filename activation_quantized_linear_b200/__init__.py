@@ -1,0 +1,288 @@
+"""ConvRot int8_tensorwise linear layer on NVIDIA B200 (sm_100a).
+
+A thin ctypes binding over libconvrot.so (C ABI in include/convrot.h).  Torch
+provides device memory and the current stream only; every step of the layer
+runs in the library's CUDA kernels.  There is no CPU fallback: if the library
+is missing, importing the binding raises.
+
+Entry points (same names as the C ABI, without the `convrot_` prefix):
+    Rotation(R)                               the G x G rotation block, on the current device
+    quantize_weight(W, rot)          -> (Wq, s_w)
+    dequant_derotate(Wq, s_w, rot)   -> W_hat (bf16)
+    rotate_quant_act(x, rot)         -> (xq, s_tok)
+    int8_gemm(xq, s_tok, Wq, s_w, bias)      -> y (bf16)
+    int8_gemm_s32(xq, Wq)                    -> acc (int32)
+    linear_int8(x, Wq, s_w, rot, bias)       -> y (bf16)
+    workspace_bytes(M, N, K), check_status()
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+import torch
+
+from . import build as _build
+
+__all__ = [
+    "ConvRotError", "Rotation", "quantize_weight", "dequant_derotate", "rotate_quant_act",
+    "int8_gemm", "int8_gemm_s32", "linear_int8", "workspace_bytes", "check_status",
+    "device_supported", "library_path", "ConvRotLinear",
+]
+
+OK, INVALID_ARG, UNSUPPORTED, CUDA, WORKSPACE, TIMEOUT, ALIGNMENT = range(7)
+OP_LINEAR_INT8 = 1
+STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "CUDA", 4: "WORKSPACE",
+                5: "TIMEOUT", 6: "ALIGNMENT"}
+
+
+class ConvRotError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"convrot {STATUS_NAMES.get(status, status)}: {message}")
+        self.status = status
+
+
+def library_path() -> str:
+    return _build.LIB_PATH
+
+
+def _load() -> ctypes.CDLL:
+    path = _build.LIB_PATH
+    if not os.path.exists(path):
+        raise ImportError(
+            f"{path} is missing: build it with `python -m activation_quantized_linear_b200.build`"
+            " (the layer has no CPU fallback)")
+    lib = ctypes.CDLL(path)
+    vp, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+    sigs = {
+        "convrot_version": ([], i32),
+        "convrot_device_supported": ([i32], i32),
+        "convrot_last_error_string": ([], ctypes.c_char_p),
+        "convrot_rotation_create": ([vp, i32, ctypes.POINTER(vp)], i32),
+        "convrot_rotation_destroy": ([vp], i32),
+        "convrot_rotation_info": ([vp, ctypes.POINTER(i32), ctypes.POINTER(i32)], i32),
+        "convrot_quantize_weight": ([vp, i64, i64, vp, vp, vp, vp], i32),
+        "convrot_dequant_derotate": ([vp, vp, i64, i64, i64, vp, vp, vp], i32),
+        "convrot_rotate_quant_act": ([vp, i64, i64, vp, vp, vp, vp], i32),
+        "convrot_int8_gemm": ([vp, vp, vp, vp, i64, vp, i64, i64, i64, vp, vp], i32),
+        "convrot_int8_gemm_s32": ([vp, vp, i64, i64, i64, vp, vp], i32),
+        "convrot_linear_int8": ([vp, i64, i64, i64, vp, vp, vp, i64, vp, vp, vp, sz, vp], i32),
+        "convrot_workspace_bytes": ([i32, i64, i64, i64], sz),
+        "convrot_check_status": ([vp], i32),
+    }
+    for name, (args, res) in sigs.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = res
+    return lib
+
+
+_lib = _load()
+
+
+def _check(status: int) -> None:
+    if status != OK:
+        raise ConvRotError(status, _lib.convrot_last_error_string().decode())
+
+
+def _stream() -> int:
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _ptr(t: torch.Tensor | None) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _need(t: torch.Tensor, name: str, dtype: torch.dtype, ndim: int) -> None:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dimensions, got shape {tuple(t.shape)}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def device_supported(device: int = 0) -> bool:
+    return bool(_lib.convrot_device_supported(device))
+
+
+class Rotation:
+    """The orthogonal G x G block R (float32), copied to the current device.
+
+    A normalized Sylvester-Hadamard R (bit for bit) selects the butterfly
+    kernels; any other orthogonal R the dense ones."""
+
+    def __init__(self, R):
+        if isinstance(R, torch.Tensor):
+            R = R.detach().to("cpu").float().numpy()
+        R = np.ascontiguousarray(R, dtype=np.float32)
+        if R.ndim != 2 or R.shape[0] != R.shape[1]:
+            raise ValueError("R must be a square matrix")
+        self._R = R
+        h = ctypes.c_void_p()
+        _check(_lib.convrot_rotation_create(R.ctypes.data, int(R.shape[0]), ctypes.byref(h)))
+        self._h = h
+        g, syl = ctypes.c_int(), ctypes.c_int()
+        _check(_lib.convrot_rotation_info(h, ctypes.byref(g), ctypes.byref(syl)))
+        self.G = g.value
+        self.is_sylvester = bool(syl.value)
+        self.device = torch.cuda.current_device()
+
+    @property
+    def handle(self) -> ctypes.c_void_p:
+        if self._h is None:
+            raise ValueError("rotation was closed")
+        return self._h
+
+    @property
+    def matrix(self) -> np.ndarray:
+        return self._R
+
+    def close(self) -> None:
+        if getattr(self, "_h", None) is not None:
+            _lib.convrot_rotation_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def quantize_weight(W: torch.Tensor, rot: Rotation, Wq: torch.Tensor | None = None,
+                    s_w: torch.Tensor | None = None):
+    """W [N, K] bf16 -> (Wq [N, K] int8, s_w [1] float32)."""
+    _need(W, "W", torch.bfloat16, 2)
+    N, K = W.shape
+    Wq = torch.empty((N, K), dtype=torch.int8, device=W.device) if Wq is None else Wq
+    s_w = torch.empty(1, dtype=torch.float32, device=W.device) if s_w is None else s_w
+    _check(_lib.convrot_quantize_weight(_ptr(W), N, K, rot.handle, _ptr(Wq), _ptr(s_w), _stream()))
+    return Wq, s_w
+
+
+def dequant_derotate(Wq: torch.Tensor, s_w: torch.Tensor, rot: Rotation,
+                     out: torch.Tensor | None = None) -> torch.Tensor:
+    """Wq [N, K] int8, s_w [1] or [N] float32 -> W_hat [N, K] bf16."""
+    _need(Wq, "Wq", torch.int8, 2)
+    _need(s_w, "s_w", torch.float32, 1)
+    N, K = Wq.shape
+    out = torch.empty((N, K), dtype=torch.bfloat16, device=Wq.device) if out is None else out
+    _check(_lib.convrot_dequant_derotate(_ptr(Wq), _ptr(s_w), s_w.numel(), N, K, rot.handle,
+                                         _ptr(out), _stream()))
+    return out
+
+
+def rotate_quant_act(x: torch.Tensor, rot: Rotation, xq: torch.Tensor | None = None,
+                     s_tok: torch.Tensor | None = None):
+    """x [M, K] bf16 -> (xq [M, K] int8, s_tok [M] float32)."""
+    _need(x, "x", torch.bfloat16, 2)
+    M, K = x.shape
+    xq = torch.empty((M, K), dtype=torch.int8, device=x.device) if xq is None else xq
+    s_tok = torch.empty(M, dtype=torch.float32, device=x.device) if s_tok is None else s_tok
+    _check(_lib.convrot_rotate_quant_act(_ptr(x), M, K, rot.handle, _ptr(xq), _ptr(s_tok),
+                                         _stream()))
+    return xq, s_tok
+
+
+def int8_gemm(xq: torch.Tensor, s_tok: torch.Tensor, Wq: torch.Tensor, s_w: torch.Tensor,
+              bias: torch.Tensor | None = None, out: torch.Tensor | None = None) -> torch.Tensor:
+    """y = bf16(xq . Wq^T * s_tok[:, None] * s_w + bias)."""
+    _need(xq, "xq", torch.int8, 2)
+    _need(Wq, "Wq", torch.int8, 2)
+    _need(s_tok, "s_tok", torch.float32, 1)
+    _need(s_w, "s_w", torch.float32, 1)
+    if bias is not None:
+        _need(bias, "bias", torch.bfloat16, 1)
+    M, K = xq.shape
+    N = Wq.shape[0]
+    if Wq.shape[1] != K:
+        raise ValueError("xq and Wq disagree on K")
+    out = torch.empty((M, N), dtype=torch.bfloat16, device=xq.device) if out is None else out
+    _check(_lib.convrot_int8_gemm(_ptr(xq), _ptr(s_tok), _ptr(Wq), _ptr(s_w), s_w.numel(),
+                                  _ptr(bias), M, N, K, _ptr(out), _stream()))
+    return out
+
+
+def int8_gemm_s32(xq: torch.Tensor, Wq: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
+    """acc = xq . Wq^T as int32 (diagnostic form of the GEMM)."""
+    _need(xq, "xq", torch.int8, 2)
+    _need(Wq, "Wq", torch.int8, 2)
+    M, K = xq.shape
+    N = Wq.shape[0]
+    if Wq.shape[1] != K:
+        raise ValueError("xq and Wq disagree on K")
+    out = torch.empty((M, N), dtype=torch.int32, device=xq.device) if out is None else out
+    _check(_lib.convrot_int8_gemm_s32(_ptr(xq), _ptr(Wq), M, N, K, _ptr(out), _stream()))
+    return out
+
+
+def workspace_bytes(M: int, N: int, K: int) -> int:
+    return int(_lib.convrot_workspace_bytes(OP_LINEAR_INT8, M, N, K))
+
+
+def linear_int8(x: torch.Tensor, Wq: torch.Tensor, s_w: torch.Tensor, rot: Rotation,
+                bias: torch.Tensor | None = None, out: torch.Tensor | None = None,
+                workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """The int8-compute forward: rotate+quantize x per token, int8 GEMM, rescale."""
+    _need(x, "x", torch.bfloat16, 2)
+    _need(Wq, "Wq", torch.int8, 2)
+    _need(s_w, "s_w", torch.float32, 1)
+    if bias is not None:
+        _need(bias, "bias", torch.bfloat16, 1)
+    M, K = x.shape
+    N = Wq.shape[0]
+    need = workspace_bytes(M, N, K)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=x.device)
+    out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device) if out is None else out
+    _check(_lib.convrot_linear_int8(_ptr(x), M, K, N, rot.handle, _ptr(Wq), _ptr(s_w), s_w.numel(),
+                                    _ptr(bias), _ptr(out), _ptr(workspace), workspace.numel(),
+                                    _stream()))
+    return out
+
+
+def check_status(stream: torch.cuda.Stream | None = None) -> None:
+    """Synchronize and raise if a kernel gave up a bounded wait since the last check."""
+    s = (stream or torch.cuda.current_stream()).cuda_stream
+    _check(_lib.convrot_check_status(s))
+
+
+class ConvRotLinear:
+    """A ConvRot int8_tensorwise linear: int8 weight, per-tensor scale, rotation R.
+
+    `forward` runs the int8-compute path; `decode_weight` the default path's
+    weight decode (dequantize + derotate to bf16)."""
+
+    def __init__(self, W: torch.Tensor, R, bias: torch.Tensor | None = None):
+        self.rotation = R if isinstance(R, Rotation) else Rotation(R)
+        self.Wq, self.s_w = quantize_weight(W, self.rotation)
+        self.bias = bias
+        self._ws = None
+
+    @property
+    def out_features(self) -> int:
+        return self.Wq.shape[0]
+
+    @property
+    def in_features(self) -> int:
+        return self.Wq.shape[1]
+
+    def decode_weight(self, out: torch.Tensor | None = None) -> torch.Tensor:
+        return dequant_derotate(self.Wq, self.s_w, self.rotation, out=out)
+
+    def forward(self, x: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
+        M = x.shape[0]
+        need = workspace_bytes(M, self.out_features, self.in_features)
+        if self._ws is None or self._ws.numel() < need:
+            self._ws = torch.empty(max(need, 1), dtype=torch.uint8, device=x.device)
+        return linear_int8(x, self.Wq, self.s_w, self.rotation, self.bias, out=out,
+                           workspace=self._ws)
+
+    __call__ = forward

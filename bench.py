@@ -1,0 +1,428 @@
+"""Benchmark of the ConvRot int8 linear layer on B200.
+
+One step = the int8-compute forward (rotate + per-token int8 quantize, int8
+GEMM with the fused rescale/bias epilogue) of every linear of the workload, on
+inputs resident in HBM.  The headline value is int8 linear TOPS,
+sum(2 M N K) / step time.  The default path's weight decode (dequantize +
+derotate) of the same weights is timed in the same run and reported under
+"derotate".
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+  python bench.py --impl reference ...   # the CPU oracle on the host cores
+
+Multi-GPU runs (torchrun, one process per GPU) are weak-scaled replicas: each
+rank runs the whole workload on its own tokens; the layer needs no exchange, so
+there is no collective on the data path.  Time is the max over ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+MEASURED_PEAKS = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+INT8_PER_BF16 = 2.0  # nominal dense int8 : bf16 tensor throughput (4.5 : 2.25 POPS)
+
+# DRAM bytes per launch from ncu (dram__bytes_read.sum + dram__bytes_write.sum),
+# keyed by kernel and shape, valid only for the kernel source they were taken on.
+NCU_TRAFFIC = {}
+NCU_TRAFFIC_SOURCE_SHA = {}
+
+
+def source_sha(rel: str) -> str:
+    with open(os.path.join(ROOT, rel), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def load_peaks():
+    try:
+        with open(MEASURED_PEAKS) as f:
+            p = json.load(f)
+        return (float(p["hbm_gbs"]), float(p["bf16_tflops"]),
+                float(p.get("bf16_tflops_sustained", p["bf16_tflops"])), "measured")
+    except Exception:
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        try:
+            with open(self.path) as f:
+                for line in f:
+                    parts = [p.strip() for p in line.split(",")]
+                    if len(parts) >= 9:
+                        rows.append(parts)
+        except Exception:
+            pass
+        finally:
+            if self.path and os.path.exists(self.path):
+                os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing
+# ---------------------------------------------------------------------------
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1 and n_gpus != world:
+        raise SystemExit(f"--gpus {n_gpus} but WORLD_SIZE={world}")
+    return world, rank, local
+
+
+def init_pg(world: int, backend: str):
+    import datetime
+
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def max_over_ranks(value: float, world: int, device) -> float:
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ---------------------------------------------------------------------------
+# CPU baseline: the oracle on a bounded sample of the same workload
+# ---------------------------------------------------------------------------
+def oracle_sample_rate(lins, rows_per_linear: int, budget_s: float):
+    """int8 linear TOPS of the oracle (rotate+quantize, GEMM, epilogue) on
+    `rows_per_linear` tokens of each linear, repeated until `budget_s`."""
+    import oracle
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        cores = os.cpu_count() or 1
+    prepared = []
+    for i, lin in enumerate(lins):
+        inp = workloads.make_layer_inputs(lin, 1, M=rows_per_linear)
+        Wq, s_w = oracle.quantize_weight(inp.W, inp.R)
+        prepared.append((lin, inp, Wq, s_w))
+    ops = 0.0
+    t0 = time.perf_counter()
+    reps = 0
+    while True:
+        for lin, inp, Wq, s_w in prepared:
+            oracle.linear_int8(inp.x, Wq, s_w, inp.R, inp.bias)
+            ops += 2.0 * rows_per_linear * lin.N * lin.K
+        reps += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return ops / dt / 1e12, cores, dt, reps
+
+
+def run_reference(args, lins):
+    world, rank, local = dist_setup(args.gpus)
+    if rank != 0:
+        return 0
+    rows = args.ref_rows
+    step_s = []
+    rates = []
+    cores = 1
+    for k in range(args.warmup + args.steps):
+        tops, cores, dt, _ = oracle_sample_rate(lins, rows, budget_s=0.0)
+        if k >= args.warmup:
+            step_s.append(dt)
+            rates.append(tops)
+    value = statistics.mean(rates)
+    sample = (f"{rows} tokens of each of the {len(lins)} linears of {args.workload} "
+              f"per step (rotate+quantize, int8 GEMM, epilogue; float64 numpy)")
+    line = {
+        "impl": "reference", "metric": "int8 ConvRot linear TOPS (rotate+quant+GEMM)",
+        "value": value, "unit": "TOPS", "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * statistics.mean(step_s),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": config_dict(args, lins),
+        "cpu_baseline": {"value": value, "unit": "TOPS", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+    return 0
+
+
+def config_dict(args, lins):
+    return {
+        "workload": args.workload,
+        "linears": [f"{l.name}:M{l.M}xK{l.K}->N{l.N}" for l in lins],
+        "G": lins[0].G, "rotation": "sylvester-hadamard",
+        "l2": "flushed between timed steps (256 MiB write + 256 MiB read, untimed)",
+    }
+
+
+# ---------------------------------------------------------------------------
+# the GPU arm
+# ---------------------------------------------------------------------------
+def run_ours(args, lins):
+    import torch
+
+    world, rank, local = dist_setup(args.gpus)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    init_pg(world, "nccl")
+    import activation_quantized_linear_b200 as cr
+
+    hbm_gbs, bf16_tflops, bf16_sust, peak_src = load_peaks()
+    int8_peak = bf16_tflops * INT8_PER_BF16
+
+    rot = cr.Rotation(workloads.sylvester_rotation(lins[0].G))
+    layers = []
+    for i, lin in enumerate(lins):
+        inp = workloads.make_layer_inputs(lin, 1 + rank)  # every rank its own tokens
+        W = inp.W.to(dev)
+        Wq, s_w = cr.quantize_weight(W, rot)
+        del W
+        layers.append(dict(
+            lin=lin, x=inp.x.to(dev), x_host=inp.x.pin_memory(), Wq=Wq, s_w=s_w,
+            bias=inp.bias.to(dev),
+            xq=torch.empty((lin.M, lin.K), dtype=torch.int8, device=dev),
+            s_tok=torch.empty(lin.M, dtype=torch.float32, device=dev),
+            y=torch.empty((lin.M, lin.N), dtype=torch.bfloat16, device=dev),
+            y_host=torch.empty((lin.M, lin.N), dtype=torch.bfloat16).pin_memory(),
+            W_hat=torch.empty((lin.N, lin.K), dtype=torch.bfloat16, device=dev),
+            ws=torch.empty(cr.workspace_bytes(lin.M, lin.N, lin.K), dtype=torch.uint8,
+                           device=dev),
+        ))
+    # L2 flush between timed steps: write 256 MiB (evicts everything), then read
+    # another 256 MiB so that the dirty flush lines are written back before the
+    # next step starts rather than during its first kernel.
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush_rd = torch.ones(64 << 20, dtype=torch.float32, device=dev)
+
+    def flush_l2(k):
+        flush.fill_(k & 0xFF)
+        flush_rd.sum()
+    stream = torch.cuda.current_stream()
+    n_lin = len(layers)
+
+    def ev():
+        return torch.cuda.Event(enable_timing=True)
+
+    def step(record):
+        for i, L in enumerate(layers):
+            e0, e1, e2 = record[i]
+            e0.record(stream)
+            cr.rotate_quant_act(L["x"], rot, xq=L["xq"], s_tok=L["s_tok"])
+            e1.record(stream)
+            cr.int8_gemm(L["xq"], L["s_tok"], L["Wq"], L["s_w"], L["bias"], out=L["y"])
+            e2.record(stream)
+
+    # ---------------- warm-up
+    for _ in range(args.warmup):
+        step([(ev(), ev(), ev()) for _ in range(n_lin)])
+    torch.cuda.synchronize()
+    cr.check_status()
+
+    # ---------------- timed: int8-compute forward
+    recs = [[(ev(), ev(), ev()) for _ in range(n_lin)] for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        for k in range(args.steps):
+            flush_l2(k)
+            step(recs[k])
+        torch.cuda.synchronize()
+    barrier(world)
+    cr.check_status()
+    clk = clocks.summary()
+
+    rqa_ms = np.array([[r[i][0].elapsed_time(r[i][1]) for i in range(n_lin)] for r in recs])
+    gemm_ms = np.array([[r[i][1].elapsed_time(r[i][2]) for i in range(n_lin)] for r in recs])
+    step_ms = np.array([r[0][0].elapsed_time(r[-1][2]) for r in recs])
+    local_total_ms = float(step_ms.sum())
+    total_ms = max_over_ranks(local_total_ms, world, dev)
+    ops_step = sum(2.0 * L["lin"].M * L["lin"].N * L["lin"].K for L in layers)
+    value = ops_step * args.steps * world / (total_ms * 1e-3) / 1e12
+
+    gemm_mean = gemm_ms.mean(axis=0)
+    gemm_ops = np.array([2.0 * L["lin"].M * L["lin"].N * L["lin"].K for L in layers])
+    gemm_tops = float(gemm_ops.sum() / (gemm_mean.sum() * 1e-3) / 1e12)
+    rqa_mean = rqa_ms.mean(axis=0)
+    rqa_bytes = np.array([3.0 * L["lin"].M * L["lin"].K + 4.0 * L["lin"].M for L in layers])
+    rqa_gbs = float(rqa_bytes.sum() / (rqa_mean.sum() * 1e-3) / 1e9)
+
+    gemm_src = "activation_quantized_linear_b200/csrc/int8_gemm.cu"
+    traffic = None
+    key = "int8_gemm_tcgen05"
+    if NCU_TRAFFIC.get(key) and NCU_TRAFFIC_SOURCE_SHA.get(key) == source_sha(gemm_src):
+        traffic = NCU_TRAFFIC[key]
+
+    # ---------------- timed: default-path weight decode (dequant + derotate)
+    drecs = [[(ev(), ev()) for _ in range(n_lin)] for _ in range(args.steps)]
+    for L in layers:
+        cr.dequant_derotate(L["Wq"], L["s_w"], rot, out=L["W_hat"])
+    torch.cuda.synchronize()
+    for k in range(args.steps):
+        flush_l2(k)
+        for i, L in enumerate(layers):
+            drecs[k][i][0].record(stream)
+            cr.dequant_derotate(L["Wq"], L["s_w"], rot, out=L["W_hat"])
+            drecs[k][i][1].record(stream)
+    torch.cuda.synchronize()
+    der_ms = np.array([[r[i][0].elapsed_time(r[i][1]) for i in range(n_lin)] for r in drecs])
+    der_bytes = np.array([3.0 * L["lin"].N * L["lin"].K for L in layers])
+    der_gbs = float(der_bytes.sum() / (der_ms.mean(axis=0).sum() * 1e-3) / 1e9)
+
+    # ---------------- end to end through the public API with host buffers
+    h2d = sum(L["x_host"].numel() * 2 for L in layers)
+    d2h = sum(L["y_host"].numel() * 2 for L in layers)
+    e2e_ms = []
+    for k in range(max(2, min(args.steps, 5)) + 1):
+        flush_l2(k)
+        e0, e1 = ev(), ev()
+        e0.record(stream)
+        for L in layers:
+            L["x"].copy_(L["x_host"], non_blocking=True)
+            cr.linear_int8(L["x"], L["Wq"], L["s_w"], rot, L["bias"], out=L["y"], workspace=L["ws"])
+            L["y_host"].copy_(L["y"], non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if k:  # first pass warms the pinned-copy path
+            e2e_ms.append(e0.elapsed_time(e1))
+    e2e_total = max_over_ranks(float(np.mean(e2e_ms)), world, dev)
+    e2e_value = ops_step * world / (e2e_total * 1e-3) / 1e12
+
+    if rank != 0:
+        return 0
+    tops_frac = gemm_tops / int8_peak
+    out = {
+        "metric": "int8 ConvRot linear TOPS (rotate+quant+GEMM)",
+        "value": value, "unit": "TOPS", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "int8", "data": "synthetic", "config": config_dict(args, lins),
+        "roofline": {
+            "kernel": "int8_gemm_tcgen05", "bound": "tensor", "achieved": gemm_tops,
+            "peak": int8_peak, "unit": "TFLOP/s", "frac": tops_frac, "traffic": traffic,
+            "peak_source": f"{peak_src} bf16 {bf16_tflops} TFLOP/s (burst) x {INT8_PER_BF16} "
+                           f"nominal int8:bf16",
+        },
+        "kernels": {
+            "rotate_quant_act": {"ms": rqa_mean.tolist(), "GB/s": rqa_gbs,
+                                 "frac_hbm": rqa_gbs / hbm_gbs},
+            "int8_gemm": {"ms": gemm_mean.tolist(), "TOPS": gemm_tops, "frac_int8_peak": tops_frac},
+        },
+        "derotate": {"metric": "dequant+derotate GB/s", "value": der_gbs, "unit": "GB/s",
+                     "ms": der_ms.mean(axis=0).tolist(), "peak": hbm_gbs,
+                     "frac": der_gbs / hbm_gbs, "bytes_per_element": 3},
+        "e2e": {"value": e2e_value, "unit": "TOPS", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_total},
+        "gpu_launches": 2 * n_lin * args.steps,
+        "clocks": clk,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        tops, cores, dt, reps = oracle_sample_rate(lins, args.ref_rows, budget_s=args.cpu_budget)
+        out["cpu_baseline"] = {
+            "value": tops, "unit": "TOPS", "cores": cores, "kind": "oracle",
+            "sample": f"{args.ref_rows} tokens of each linear, {reps} passes in {dt:.1f} s "
+                      f"(rotate+quantize, int8 GEMM, epilogue; float64 numpy)"}
+    print(json.dumps(out))
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="zimage_dit_block",
+                    choices=[k for k in workloads.WORKLOADS if k != "group_size_sweep"])
+    ap.add_argument("--ref-rows", type=int, default=64)
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    lins = workloads.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, lins)
+    try:
+        return run_ours(args, lins)
+    finally:
+        try:
+            import torch.distributed as dist
+            if dist.is_initialized():
+                dist.destroy_process_group()
+        except Exception:
+            pass
+
+
+if __name__ == "__main__":
+    sys.exit(main())

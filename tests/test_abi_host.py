@@ -1,0 +1,116 @@
+"""Host-side checks of the C ABI (no kernel launch; runs without a GPU).
+
+The library must load on a machine without a GPU, export every entry point
+include/convrot.h declares, and reject bad arguments with the documented
+status before touching the device.
+"""
+
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import activation_quantized_linear_b200 as cr
+from activation_quantized_linear_b200 import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "convrot.h")
+
+lib = cr._lib
+vp = ctypes.c_void_p
+FAKE = 0x10000          # a 16-byte aligned address that is never dereferenced
+MISALIGNED = 0x10008
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(convrot_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_function():
+    names = declared_functions()
+    assert len(names) >= 14
+    raw = ctypes.CDLL(build.LIB_PATH)
+    for n in names:
+        assert hasattr(raw, n), f"{n} declared in convrot.h but not exported"
+
+
+def test_version_and_error_string():
+    assert lib.convrot_version() >= 100
+    assert isinstance(lib.convrot_last_error_string(), bytes)
+
+
+@pytest.mark.parametrize("G", [0, 1, 2, 8, 32, 128, 512, -4])
+def test_rotation_rejects_group_size(G):
+    R = np.eye(max(G, 1), dtype=np.float32)
+    h = vp()
+    st = lib.convrot_rotation_create(R.ctypes.data, G, ctypes.byref(h))
+    assert st == cr.UNSUPPORTED
+    assert h.value is None
+    assert b"group size" in lib.convrot_last_error_string()
+
+
+def test_rotation_rejects_non_orthogonal_and_null():
+    h = vp()
+    R = np.eye(16, dtype=np.float32)
+    R[0, 1] = 0.01
+    assert lib.convrot_rotation_create(R.ctypes.data, 16, ctypes.byref(h)) == cr.INVALID_ARG
+    assert b"orthogonal" in lib.convrot_last_error_string()
+    assert lib.convrot_rotation_create(None, 16, ctypes.byref(h)) == cr.INVALID_ARG
+    assert lib.convrot_rotation_create(R.ctypes.data, 16, None) == cr.INVALID_ARG
+
+
+def test_null_handle_rejected():
+    assert lib.convrot_rotation_destroy(None) == cr.INVALID_ARG
+    assert lib.convrot_rotate_quant_act(FAKE, 4, 256, None, FAKE, FAKE, None) == cr.INVALID_ARG
+    assert lib.convrot_dequant_derotate(FAKE, FAKE, 1, 4, 256, None, FAKE, None) == cr.INVALID_ARG
+    assert lib.convrot_quantize_weight(FAKE, 4, 256, None, FAKE, FAKE, None) == cr.INVALID_ARG
+
+
+def test_gemm_shape_and_pointer_checks():
+    g = lib.convrot_int8_gemm
+    # N not a multiple of 16, K not a multiple of 16, negative M
+    assert g(FAKE, FAKE, FAKE, FAKE, 1, None, 8, 24, 64, FAKE, None) == cr.INVALID_ARG
+    assert g(FAKE, FAKE, FAKE, FAKE, 1, None, 8, 32, 40, FAKE, None) == cr.INVALID_ARG
+    assert g(FAKE, FAKE, FAKE, FAKE, 1, None, -1, 32, 64, FAKE, None) == cr.INVALID_ARG
+    assert g(FAKE, FAKE, FAKE, FAKE, 1, None, 8, 32, 1 << 20, FAKE, None) == cr.UNSUPPORTED
+    # M == 0 is a no-op that never touches the pointers
+    assert g(None, None, None, None, 1, None, 0, 32, 64, None, None) == cr.OK
+    # null / misaligned operands
+    assert g(None, FAKE, FAKE, FAKE, 1, None, 8, 32, 64, FAKE, None) == cr.INVALID_ARG
+    assert g(MISALIGNED, FAKE, FAKE, FAKE, 1, None, 8, 32, 64, FAKE, None) == cr.ALIGNMENT
+    assert g(FAKE, FAKE, MISALIGNED, FAKE, 1, None, 8, 32, 64, FAKE, None) == cr.ALIGNMENT
+    assert g(FAKE, FAKE, FAKE, FAKE, 1, None, 8, 32, 64, MISALIGNED, None) == cr.ALIGNMENT
+    assert g(FAKE, None, FAKE, FAKE, 1, None, 8, 32, 64, FAKE, None) == cr.INVALID_ARG
+    # scale length must be 1 or N
+    assert g(FAKE, FAKE, FAKE, FAKE, 3, None, 8, 32, 64, FAKE, None) == cr.INVALID_ARG
+    assert g(FAKE, FAKE, FAKE, FAKE, 1, MISALIGNED, 8, 32, 64, FAKE, None) == cr.ALIGNMENT
+    s = lib.convrot_int8_gemm_s32
+    assert s(FAKE, FAKE, 8, 20, 64, FAKE, None) == cr.INVALID_ARG
+    assert s(FAKE, FAKE, 0, 32, 64, None, None) == cr.OK
+
+
+def test_workspace_size():
+    M, N, K = 4608, 11520, 3840
+    need = lib.convrot_workspace_bytes(cr.OP_LINEAR_INT8, M, N, K)
+    assert need >= M * K + 4 * M and need % 256 == 0
+    assert lib.convrot_workspace_bytes(99, M, N, K) == 0
+    assert lib.convrot_workspace_bytes(cr.OP_LINEAR_INT8, 0, N, K) == 0
+
+
+def test_linear_rejects_before_device():
+    f = lib.convrot_linear_int8
+    assert f(FAKE, 8, 256, 24, None, FAKE, FAKE, 1, None, FAKE, FAKE, 1 << 20, None) == cr.INVALID_ARG
+    assert f(FAKE, 8, 256, 32, None, FAKE, FAKE, 1, None, FAKE, FAKE, 1 << 20, None) == cr.INVALID_ARG
+
+
+def test_binding_validates_tensors_on_cpu():
+    import torch
+    x = torch.zeros(4, 256, dtype=torch.float32)
+    with pytest.raises(TypeError):
+        cr.rotate_quant_act(x, None)
+    with pytest.raises(ValueError):
+        cr.rotate_quant_act(x.to(torch.bfloat16), None)  # not a CUDA tensor

@@ -1,0 +1,301 @@
+"""Per-kernel parity of the CUDA path against the CPU oracle on small and odd
+shapes (several tiles plus ragged tails), through the C ABI.
+
+Tolerances (fixed by the acceptance criteria of the layer):
+  * int32 accumulators: bit-exact given identical int8 codes;
+  * activation / weight codes: at most 1 LSB apart on at most 0.1 % of the
+    elements (float32 rotation order and reciprocal-vs-division at .5 ties);
+  * scales: relative 1e-6;
+  * derotated bf16 weight: bit-exact for the Sylvester R (exact integer sums and
+    a single correct rounding), within 1 bf16 ulp for a dense R;
+  * layer output: relative L2 <= 2e-3 against the oracle, and cosine >= 0.999
+    against the unquantized float64 layer.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from tests._gpu_helpers import (Guarded, assert_codes_close, bf16_bits, bf16_ulp,
+                                to_cuda_bf16)
+
+pytestmark = pytest.mark.gpu
+
+cr = None
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    global cr
+    import activation_quantized_linear_b200 as mod
+    cr = mod
+    torch.cuda.set_device(0)
+    assert mod.device_supported(0), "these kernels are built for sm_100a (B200)"
+    yield
+
+
+def _rotation(G, kind):
+    return workloads.sylvester_rotation(G) if kind == "sylvester" else workloads.qr_rotation(G, seed=6000 + G)
+
+
+def _scale_rtol(G, kind):
+    """Relative tolerance of a float32 absmax scale against the float64 oracle.
+    The butterfly adds exact-sign terms with a few roundings: 1e-6.  A dense R
+    sums G float32 products: the classic bound G * 2^-24 of a float32 dot product."""
+    return 1e-6 if kind == "sylvester" else G * 2.0 ** -24
+
+
+def _codes(rng, shape):
+    return rng.integers(-127, 128, size=shape, dtype=np.int64).astype(np.int8)
+
+
+# ---------------------------------------------------------------------------
+# int8 GEMM main loop: bit-exact int32
+# ---------------------------------------------------------------------------
+GEMM_SHAPES = [
+    (1, 16, 16), (7, 144, 64), (128, 256, 128), (129, 272, 144), (257, 512, 1024),
+    (300, 1024, 3840), (64, 1024, 1024), (1000, 528, 2048), (33, 4096, 256),
+]
+
+
+@pytest.mark.parametrize("M,N,K", GEMM_SHAPES)
+def test_int8_gemm_s32_bit_exact(M, N, K):
+    rng = np.random.default_rng(M * 7 + N * 3 + K)
+    a = _codes(rng, (M, K))
+    b = _codes(rng, (N, K))
+    out = Guarded((M, N), torch.int32)
+    acc = cr.int8_gemm_s32(torch.from_numpy(a).cuda(), torch.from_numpy(b).cuda(), out=out.tensor)
+    torch.cuda.synchronize()
+    out.check()
+    np.testing.assert_array_equal(acc.cpu().numpy(), oracle.int8_gemm_acc(a, b))
+
+
+def test_int8_gemm_s32_extremes():
+    """Largest accumulators of the workloads (|acc| = 127^2 K, K = 15360)."""
+    K = 15360
+    a = np.full((130, K), 127, np.int8)
+    a[1::2] = -127
+    a[5, ::2] = 0
+    b = np.full((272, K), 127, np.int8)
+    b[3] = -127
+    b[7, :100] = 0
+    acc = cr.int8_gemm_s32(torch.from_numpy(a).cuda(), torch.from_numpy(b).cuda())
+    ref = oracle.int8_gemm_acc(a, b)
+    assert abs(int(ref[0, 0])) == 127 * 127 * K
+    np.testing.assert_array_equal(acc.cpu().numpy(), ref)
+
+
+def test_int8_gemm_deterministic():
+    rng = np.random.default_rng(11)
+    a = torch.from_numpy(_codes(rng, (777, 3072))).cuda()
+    b = torch.from_numpy(_codes(rng, (1280, 3072))).cuda()
+    s_tok = torch.rand(777, device="cuda") * 0.01
+    s_w = torch.tensor([1e-3], device="cuda")
+    bias = torch.randn(1280, device="cuda").to(torch.bfloat16)
+    y1 = cr.int8_gemm(a, s_tok, b, s_w, bias)
+    y2 = cr.int8_gemm(a, s_tok, b, s_w, bias)
+    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+
+
+# ---------------------------------------------------------------------------
+# int8 GEMM epilogue: rescale + bias -> bf16
+# ---------------------------------------------------------------------------
+def _assert_epilogue_close(y_gpu, acc, s_tok, s_w, bias):
+    ref = oracle.epilogue(acc, s_tok, s_w if np.ndim(s_w) == 0 else 1.0, bias)
+    if np.ndim(s_w) == 1:  # per output channel
+        y64 = (acc.astype(np.float64) * s_tok.astype(np.float64)[:, None]
+               * s_w.astype(np.float64)[None, :])
+        if bias is not None:
+            y64 = y64 + oracle.as_f64(bias)[None, :]
+        ref = oracle.bf16_round(y64)
+    got = oracle.as_f64(y_gpu)
+    mag = np.abs(acc.astype(np.float64) * s_tok.astype(np.float64)[:, None]
+                 * np.abs(np.asarray(s_w, np.float64)).max())
+    if bias is not None:
+        mag = mag + np.abs(oracle.as_f64(bias))[None, :]
+    tol = bf16_ulp(ref) + mag * 2.0 ** -21
+    bad = np.abs(got - ref) > tol
+    assert not bad.any(), f"{bad.sum()} epilogue outputs off by more than 1 ulp"
+
+
+@pytest.mark.parametrize("M,N,K,with_bias,per_channel", [
+    (64, 1024, 1024, True, False), (129, 272, 144, False, False), (7, 144, 64, True, True),
+    (257, 512, 256, True, True),
+])
+def test_int8_gemm_epilogue(M, N, K, with_bias, per_channel):
+    rng = np.random.default_rng(M + N + K)
+    a = _codes(rng, (M, K))
+    b = _codes(rng, (N, K))
+    s_tok = (rng.random(M) * 0.05).astype(np.float32)
+    s_tok[0] = 0.0  # a zero token: output row = bias
+    s_w = (rng.random(N) * 2e-3 + 1e-4).astype(np.float32) if per_channel else np.float32(1.3e-3)
+    bias = workloads.to_bf16(rng.standard_normal(N).astype(np.float32) * 0.5) if with_bias else None
+    out = Guarded((M, N), torch.bfloat16)
+    y = cr.int8_gemm(torch.from_numpy(a).cuda(), torch.from_numpy(s_tok).cuda(),
+                     torch.from_numpy(b).cuda(), torch.from_numpy(np.atleast_1d(s_w)).cuda(),
+                     bias.cuda() if bias is not None else None, out=out.tensor)
+    torch.cuda.synchronize()
+    out.check()
+    acc = oracle.int8_gemm_acc(a, b)
+    _assert_epilogue_close(y.cpu(), acc, s_tok, s_w, bias)
+    if with_bias:
+        np.testing.assert_array_equal(oracle.as_f64(y[0].cpu()), oracle.as_f64(bias))
+
+
+# ---------------------------------------------------------------------------
+# activation rotate + quantize
+# ---------------------------------------------------------------------------
+RQA_CASES = [
+    (G, kind, M, K)
+    for G in (4, 16, 64, 256) for kind in ("sylvester", "qr")
+    for (M, K) in ((1, 256), (7, 1024), (129, 3840))
+] + [(256, "sylvester", 33, 15360), (256, "sylvester", 17, 32768), (64, "sylvester", 20, 12288),
+     (256, "qr", 9, 10240), (16, "sylvester", 65, 5120), (256, "sylvester", 300, 2048)]
+
+
+@pytest.mark.parametrize("G,kind,M,K", RQA_CASES)
+def test_rotate_quant_act_parity(G, kind, M, K):
+    R = _rotation(G, kind)
+    rot = cr.Rotation(R)
+    assert rot.is_sylvester == (kind == "sylvester")
+    x = workloads.make_activation(M, K, seed=G + M + K, n_outliers=4)
+    x[min(2, M - 1)] = 0  # an all-zero token
+    xq_buf = Guarded((M, K), torch.int8)
+    s_buf = Guarded((M,), torch.float32)
+    xq, s_tok = cr.rotate_quant_act(x.cuda(), rot, xq=xq_buf.tensor, s_tok=s_buf.tensor)
+    torch.cuda.synchronize()
+    xq_buf.check()
+    s_buf.check()
+    ref_q, ref_s = oracle.rotate_quant_act(x, R)
+    np.testing.assert_allclose(s_tok.cpu().numpy(), ref_s, rtol=_scale_rtol(G, kind), atol=0)
+    assert_codes_close(xq.cpu().numpy(), ref_q)
+    assert float(s_tok[min(2, M - 1)]) == 0.0 and not xq[min(2, M - 1)].any()
+
+
+def test_rotate_quant_act_empty():
+    rot = cr.Rotation(workloads.sylvester_rotation(256))
+    x = torch.empty((0, 256), dtype=torch.bfloat16, device="cuda")
+    xq, s = cr.rotate_quant_act(x, rot)
+    assert xq.shape == (0, 256) and s.shape == (0,)
+
+
+def test_rotate_quant_act_rejects_bad_k():
+    rot = cr.Rotation(workloads.sylvester_rotation(256))
+    x = torch.zeros((4, 320), dtype=torch.bfloat16, device="cuda")  # 320 % 256 != 0
+    with pytest.raises(cr.ConvRotError) as e:
+        cr.rotate_quant_act(x, rot)
+    assert e.value.status == cr.INVALID_ARG
+    x = torch.zeros((4, 65536), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(cr.ConvRotError) as e:
+        cr.rotate_quant_act(x, rot)
+    assert e.value.status == cr.UNSUPPORTED
+
+
+# ---------------------------------------------------------------------------
+# weight quantization and dequant + derotate
+# ---------------------------------------------------------------------------
+WQ_CASES = [(G, kind, N, K) for G in (4, 16, 64, 256) for kind in ("sylvester", "qr")
+            for (N, K) in ((16, 256), (136, 1024))] + [(256, "sylvester", 1000, 3840)]
+
+
+@pytest.mark.parametrize("G,kind,N,K", WQ_CASES)
+def test_quantize_weight_parity(G, kind, N, K):
+    R = _rotation(G, kind)
+    rot = cr.Rotation(R)
+    W = workloads.make_weight(N, K, seed=N + K + G)
+    Wq, s_w = cr.quantize_weight(W.cuda(), rot)
+    ref_q, ref_s = oracle.quantize_weight(W, R)
+    np.testing.assert_allclose(s_w.cpu().numpy()[0], ref_s, rtol=_scale_rtol(G, kind))
+    assert_codes_close(Wq.cpu().numpy(), ref_q)
+
+
+@pytest.mark.parametrize("G,kind,N,K", WQ_CASES + [(256, "sylvester", 12288 // 8, 3072)])
+def test_dequant_derotate_parity(G, kind, N, K):
+    R = _rotation(G, kind)
+    rot = cr.Rotation(R)
+    W = workloads.make_weight(N, K, seed=N * 3 + K + G)
+    Wq, s_w = oracle.quantize_weight(W, R)
+    out = Guarded((N, K), torch.bfloat16)
+    W_hat = cr.dequant_derotate(torch.from_numpy(Wq).cuda(),
+                                torch.tensor([s_w], dtype=torch.float32, device="cuda"), rot,
+                                out=out.tensor)
+    torch.cuda.synchronize()
+    out.check()
+    ref = oracle.dequant_derotate(Wq, s_w, R)
+    got = oracle.as_f64(W_hat.cpu())
+    if kind == "sylvester":
+        np.testing.assert_array_equal(bf16_bits(W_hat), oracle.bf16_bits(ref))
+    else:
+        assert np.all(np.abs(got - ref) <= bf16_ulp(ref)), "more than 1 bf16 ulp"
+    # decode accuracy at the pages' group size; smaller groups spread the outlier
+    # columns over fewer entries, so their per-tensor scale is coarser
+    assert oracle.cosine(got, W) >= (0.9998 if G == 256 else 0.995)
+
+
+@pytest.mark.parametrize("kind", ["sylvester", "qr"])
+def test_dequant_derotate_per_channel_scale(kind):
+    """A scale per output channel multiplies along the OUTPUT axis (PR #194
+    fixed a broadcast that scaled the input axis: square weights decoded at corr
+    0.82).  Non-square on purpose, so a wrong axis cannot pass silently."""
+    N, K, G = 272, 512, 64
+    R = _rotation(G, kind)
+    rot = cr.Rotation(R)
+    rng = np.random.default_rng(5)
+    Wq = _codes(rng, (N, K))
+    s = (rng.random(N) * 1e-3 + 1e-4).astype(np.float32)
+    W_hat = cr.dequant_derotate(torch.from_numpy(Wq).cuda(), torch.from_numpy(s).cuda(), rot)
+    ref = oracle.bf16_round(s.astype(np.float64)[:, None]
+                            * oracle.block_rotate(Wq.astype(np.float64), R.astype(np.float64).T))
+    got = oracle.as_f64(W_hat.cpu())
+    if kind == "sylvester":
+        np.testing.assert_array_equal(got, ref)
+    else:
+        assert np.all(np.abs(got - ref) <= bf16_ulp(ref))
+
+
+# ---------------------------------------------------------------------------
+# the whole int8-compute layer
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("kind", ["sylvester", "qr"])
+@pytest.mark.parametrize("M", [64, 1, 130])
+def test_linear_int8_single_1024(kind, M):
+    lin = workloads.WORKLOADS["single_1024"][0]
+    inp = workloads.make_layer_inputs(lin, 0, rotation=kind, M=M)
+    Wq, s_w = oracle.quantize_weight(inp.W, inp.R)
+    rot = cr.Rotation(inp.R)
+    out = Guarded((M, lin.N), torch.bfloat16)
+    y = cr.linear_int8(inp.x.cuda(), torch.from_numpy(Wq).cuda(),
+                       torch.tensor([s_w], device="cuda"), rot, inp.bias.cuda(), out=out.tensor)
+    torch.cuda.synchronize()
+    out.check()
+    y_ref, *_ = oracle.linear_int8(inp.x, Wq, s_w, inp.R, inp.bias)
+    assert oracle.rel_l2(y.cpu(), y_ref) <= 2e-3
+    assert oracle.cosine(y.cpu(), oracle.linear_dense(inp.x, inp.W, inp.bias)) >= 0.999
+
+
+def test_linear_int8_workspace_errors():
+    rot = cr.Rotation(workloads.sylvester_rotation(256))
+    x = torch.zeros((8, 256), dtype=torch.bfloat16, device="cuda")
+    Wq = torch.zeros((32, 256), dtype=torch.int8, device="cuda")
+    s_w = torch.ones(1, device="cuda")
+    small = torch.empty(16, dtype=torch.uint8, device="cuda")
+    with pytest.raises(cr.ConvRotError) as e:
+        cr.linear_int8(x, Wq, s_w, rot, workspace=small)
+    assert e.value.status == cr.WORKSPACE
+
+
+def test_layer_module_two_modes_agree():
+    """int8-compute against the default path (decode + dense bf16 matmul)."""
+    lin = workloads.WORKLOADS["single_1024"][0]
+    inp = workloads.make_layer_inputs(lin, 0)
+    layer = cr.ConvRotLinear(inp.W.cuda(), inp.R, inp.bias.cuda())
+    y_int8 = layer(inp.x.cuda())
+    y_dec = torch.nn.functional.linear(inp.x.cuda().float(), layer.decode_weight().float(),
+                                       inp.bias.cuda().float())
+    assert oracle.cosine(y_int8.cpu(), y_dec.cpu()) >= 0.999
+
+
+def test_check_status_clean():
+    cr.check_status()
