@@ -29,7 +29,8 @@ from . import build as _build
 __all__ = [
     "ConvRotError", "Rotation", "quantize_weight", "dequant_derotate", "rotate_quant_act",
     "int8_gemm", "int8_gemm_s32", "linear_int8", "workspace_bytes", "check_status",
-    "device_supported", "library_path", "ConvRotLinear",
+    "device_supported", "library_path", "ConvRotLinear", "linear_int8_noalloc",
+    "noalloc_scratch_bytes",
 ]
 
 OK, INVALID_ARG, UNSUPPORTED, CUDA, WORKSPACE, TIMEOUT, ALIGNMENT = range(7)
@@ -70,6 +71,8 @@ def _load() -> ctypes.CDLL:
         "convrot_int8_gemm_s32": ([vp, vp, i64, i64, i64, vp, vp], i32),
         "convrot_linear_int8": ([vp, i64, i64, i64, vp, vp, vp, i64, vp, vp, vp, sz, vp], i32),
         "convrot_workspace_bytes": ([i32, i64, i64, i64], sz),
+        "convrot_linear_int8_noalloc": ([vp, i64, i64, i64, vp, vp, vp, i64, vp, vp, vp], i32),
+        "convrot_noalloc_scratch_bytes": ([], sz),
         "convrot_check_status": ([vp], i32),
     }
     for name, (args, res) in sigs.items():
@@ -246,6 +249,29 @@ def linear_int8(x: torch.Tensor, Wq: torch.Tensor, s_w: torch.Tensor, rot: Rotat
                                     _ptr(bias), _ptr(out), _ptr(workspace), workspace.numel(),
                                     _stream()))
     return out
+
+
+def linear_int8_noalloc(x: torch.Tensor, Wq: torch.Tensor, s_w: torch.Tensor, rot: Rotation,
+                       bias: torch.Tensor | None = None,
+                       out: torch.Tensor | None = None) -> torch.Tensor:
+    """linear_int8 for callers that cannot allocate device memory: the
+    intermediate codes and scales live in the library's static scratch
+    (noalloc_scratch_bytes() bytes per GPU).  Pass `out` to allocate nothing."""
+    _need(x, "x", torch.bfloat16, 2)
+    _need(Wq, "Wq", torch.int8, 2)
+    _need(s_w, "s_w", torch.float32, 1)
+    if bias is not None:
+        _need(bias, "bias", torch.bfloat16, 1)
+    M, K = x.shape
+    N = Wq.shape[0]
+    out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device) if out is None else out
+    _check(_lib.convrot_linear_int8_noalloc(_ptr(x), M, K, N, rot.handle, _ptr(Wq), _ptr(s_w),
+                                            s_w.numel(), _ptr(bias), _ptr(out), _stream()))
+    return out
+
+
+def noalloc_scratch_bytes() -> int:
+    return int(_lib.convrot_noalloc_scratch_bytes())
 
 
 def check_status(stream: torch.cuda.Stream | None = None) -> None:

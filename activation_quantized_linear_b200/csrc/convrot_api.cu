@@ -113,6 +113,18 @@ size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 }  // namespace
 
+namespace convrot {
+convrot_status set_last_error(convrot_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  std::vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return s;
+}
+}  // namespace convrot
+
 extern "C" {
 
 int convrot_version(void) { return 100; }

@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <cstdint>
 
+#include "convrot.h"
+
 struct convrot_rotation_s {
   int G;
   int is_sylvester;   // R == H_G / sqrt(G) bit for bit
@@ -50,6 +52,9 @@ cudaError_t launch_int8_gemm(const GemmArgs& a, cudaStream_t stream);
 
 // Reads and clears the current device's kernel status word (0 = fine).
 cudaError_t read_and_clear_status(unsigned int* status, cudaStream_t stream);
+
+// Records `fmt` as the calling thread's last error message and returns `s`.
+convrot_status set_last_error(convrot_status s, const char* fmt, ...);
 
 // Largest K the rotate+quantize kernel keeps on chip for one token.
 constexpr int64_t kMaxRotateK = 32768;

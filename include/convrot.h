@@ -156,6 +156,35 @@ convrot_status convrot_linear_int8(const convrot_bf16* x, int64_t M, int64_t K, 
                                    int64_t s_w_len, const convrot_bf16* bias, convrot_bf16* y,
                                    void* ws, size_t ws_bytes, convrot_stream_t stream);
 
+/*
+ * The int8-compute forward for callers that cannot allocate device memory.
+ * (No counterpart on the pages: this is an interface of this library only.)
+ * Callers such as a plugin inside a framework that owns all device memory and
+ * offers its extensions no scratch allocator, or a serving path that must not
+ * allocate (an allocation can synchronize the device and can fail with out of
+ * memory mid-request), have no workspace to pass to convrot_linear_int8.  This
+ * variant computes the same result with the same kernels, keeping the int8
+ * codes and per-token scales in a static device array of
+ * CONVROT_NOALLOC_SCRATCH_BYTES (32 MiB) that every GPU loading the library
+ * holds until the process exits.  It allocates nothing itself.
+ *   - Limit: round256(M*K) + round256(4*M) <= CONVROT_NOALLOC_SCRATCH_BYTES,
+ *     else CONVROT_ERR_UNSUPPORTED with a message naming both sizes.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - All calls share the array: calls that overlap on the GPU (other streams,
+ *     other host threads) race and must be serialized by the caller.  Each call
+ *     overwrites all of the scratch it reads, so nothing is carried over.
+ *   - Other arguments, limits and errors are those of convrot_linear_int8.
+ */
+#define CONVROT_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+convrot_status convrot_linear_int8_noalloc(const convrot_bf16* x, int64_t M, int64_t K, int64_t N,
+                                           convrot_rotation_t R, const int8_t* Wq,
+                                           const float* s_w, int64_t s_w_len,
+                                           const convrot_bf16* bias, convrot_bf16* y,
+                                           convrot_stream_t stream);
+/* Size of that static scratch in bytes (CONVROT_NOALLOC_SCRATCH_BYTES). */
+size_t convrot_noalloc_scratch_bytes(void);
+
 /* Bytes of workspace an operation needs (0 if none); 0 for an unknown op. */
 size_t convrot_workspace_bytes(int op, int64_t M, int64_t N, int64_t K);
 
