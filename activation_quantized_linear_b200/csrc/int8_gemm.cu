@@ -30,8 +30,6 @@
 
 namespace convrot {
 
-__device__ unsigned int g_kernel_status;  // bit 0: a bounded wait ran out
-
 namespace {
 
 constexpr int BM = 128;
@@ -60,6 +58,7 @@ struct Params {
   int m_tiles, n_tiles;
   int per_channel_scale;
   int out_s32;
+  unsigned int* status;  // device status word (bit 0: a wait ran out)
 };
 
 struct Barriers {
@@ -82,8 +81,8 @@ __device__ __forceinline__ void tile_coords(int tile, int m_tiles, int n_tiles, 
   nb = local / gm;
 }
 
-__device__ __forceinline__ void record_timeout(Barriers* bars) {
-  atomicOr(&g_kernel_status, 1u);
+__device__ __forceinline__ void record_timeout(Barriers* bars, unsigned int* status) {
+  atomicOr(status, 1u);
   *reinterpret_cast<volatile uint32_t*>(&bars->abort_flag) = 1u;
 }
 
@@ -182,7 +181,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tile_coords(tile, p.m_tiles, p.n_tiles, mb, nb);
       for (int kb = 0; kb < p.num_kb; ++kb) {
         if (!wait_bounded(&bars->empty[stage], phase ^ 1u)) {
-          record_timeout(bars);
+          record_timeout(bars, p.status);
           break;
         }
         ptx::mbar_arrive_expect_tx(&bars->full[stage], STAGE_BYTES);
@@ -211,7 +210,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int acc = local & 1;
       const uint32_t acc_phase = (local >> 1) & 1;
       if (!wait_bounded(&bars->acc_empty[acc], acc_phase ^ 1u)) {
-        record_timeout(bars);
+        record_timeout(bars, p.status);
         break;
       }
       ptx::tc_fence_after();
@@ -219,7 +218,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int kb = 0; kb < p.num_kb; ++kb) {
         if (!wait_bounded(&bars->full[stage], phase)) {
-          record_timeout(bars);
+          record_timeout(bars, p.status);
           ok = false;
           break;
         }
@@ -259,7 +258,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t acc_phase = (local >> 1) & 1;
       const bool ready = __all_sync(0xffffffffu, wait_bounded(&bars->acc_full[acc], acc_phase));
       if (!ready) {
-        if (lane == 0) record_timeout(bars);
+        if (lane == 0) record_timeout(bars, p.status);
         break;
       }
       ptx::tc_fence_after();
@@ -299,49 +298,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess) {
-      fn = reinterpret_cast<EncodeTiledFn>(ptr);
-    }
-  }
-  return fn;
-}
-
 // int8 [rows, K] row-major, box of `box_rows` x 128 bytes, 128-byte swizzle,
 // zero fill outside the tensor.
 bool encode_operand(CUtensorMap* map, const int8_t* base, int64_t rows, int64_t K, int box_rows) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
-  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K)};
-  const cuuint32_t box[2] = {static_cast<cuuint32_t>(BK), static_cast<cuuint32_t>(box_rows)};
-  const cuuint32_t estr[2] = {1, 1};
-  std::memset(map, 0, sizeof(*map));
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t*>(base), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-int sm_count() {
-  static int sms = 0;
-  if (!sms) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (sms <= 0) sms = 148;
-  }
-  return sms;
+  return encode_tma_2d(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, base, static_cast<uint64_t>(K),
+                       static_cast<uint64_t>(rows), static_cast<uint64_t>(K), BK,
+                       static_cast<uint32_t>(box_rows));
 }
 
 }  // namespace
@@ -361,6 +323,8 @@ cudaError_t launch_int8_gemm(const GemmArgs& a, cudaStream_t stream) {
     attr_set = true;
   }
   Params p;
+  cudaError_t se = status_word(&p.status);
+  if (se != cudaSuccess) return se;
   p.s_tok = a.s_tok;
   p.s_w = a.s_w;
   p.bias = a.bias;
@@ -376,21 +340,6 @@ cudaError_t launch_int8_gemm(const GemmArgs& a, cudaStream_t stream) {
   const int grid = tiles < sm_count() ? tiles : sm_count();
   int8_gemm_tcgen05<<<grid, kThreads, kSmemBytes, stream>>>(tmA, tmB, p);
   return cudaGetLastError();
-}
-
-cudaError_t read_and_clear_status(unsigned int* status, cudaStream_t stream) {
-  cudaError_t e = cudaStreamSynchronize(stream);
-  if (e != cudaSuccess) return e;
-  unsigned int v = 0;
-  e = cudaMemcpyFromSymbol(&v, g_kernel_status, sizeof(v));
-  if (e != cudaSuccess) return e;
-  if (v) {
-    const unsigned int zero = 0;
-    e = cudaMemcpyToSymbol(g_kernel_status, &zero, sizeof(zero));
-    if (e != cudaSuccess) return e;
-  }
-  *status = v;
-  return cudaSuccess;
 }
 
 }  // namespace convrot

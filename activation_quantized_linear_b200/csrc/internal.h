@@ -1,6 +1,7 @@
 // Internal declarations shared by the library's translation units.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <cstdint>
 
@@ -53,10 +54,24 @@ cudaError_t launch_int8_gemm(const GemmArgs& a, cudaStream_t stream);
 // Reads and clears the current device's kernel status word (0 = fine).
 cudaError_t read_and_clear_status(unsigned int* status, cudaStream_t stream);
 
+// Device address of the current device's kernel status word (kernels that
+// give up a bounded wait atomically OR bit 0 into it).
+cudaError_t status_word(unsigned int** ptr);
+
+// 2-D tiled TMA descriptor with 128-byte swizzle and zero fill outside the
+// tensor: `rows` rows of `inner_elems` elements, rows `row_stride_bytes` apart,
+// box of `box_rows` x `box_inner` elements.
+bool encode_tma_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base,
+                   uint64_t inner_elems, uint64_t rows, uint64_t row_stride_bytes,
+                   uint32_t box_inner, uint32_t box_rows);
+
+// Number of SMs of the current device.
+int sm_count();
+
 // Records `fmt` as the calling thread's last error message and returns `s`.
 convrot_status set_last_error(convrot_status s, const char* fmt, ...);
 
 // Largest K the rotate+quantize kernel keeps on chip for one token.
-constexpr int64_t kMaxRotateK = 32768;
+constexpr int64_t kMaxRotateK = 32768;  // 32 warps x 32 lanes x 32 elements
 
 }  // namespace convrot

@@ -7,12 +7,14 @@
 //     "How INT8 ConvRot Quantization Works").
 //
 // Two implementations of the G x G product:
-//   * R = H_G / sqrt(G) (Sylvester-Hadamard): an in-register fast Walsh-Hadamard
-//     butterfly.  A thread owns 32 consecutive elements ("a chunk"): the
-//     log2(min(G,32)) butterfly stages inside a chunk run in registers, the
-//     remaining log2(G/32) stages pair chunks of neighbouring lanes through
-//     warp shuffles.  The 1/sqrt(G) normalisation is a power of two and is
-//     folded into the scales, so it never rounds.  These kernels are HBM-bound.
+//   * R = H_G / sqrt(G) (Sylvester-Hadamard): a fast Walsh-Hadamard butterfly.
+//     A lane owns 32 consecutive elements as 16 packed float pairs and runs the
+//     butterfly stages two elements per instruction (sm_100 f32x2 arithmetic);
+//     for G = 256 the last three stages follow one exchange through shared
+//     memory, for G = 64 the last one a warp shuffle.  All loads are issued
+//     before any arithmetic and many warps stay resident.  The 1/sqrt(G) factor
+//     is a power of two folded into the scales, so it never rounds.  These
+//     kernels are HBM-bound.
 //   * any other orthogonal R: a shared-memory tiled product accumulated in
 //     float64 (2G flops per element, ALU-bound; a correctness path).  Inputs
 //     (bf16 or int8) and R (float32) are exact in float64, so each output is
@@ -27,7 +29,8 @@
 namespace convrot {
 namespace {
 
-constexpr int kChunk = 32;                 // elements one thread owns
+constexpr int kVec = 32;                   // elements one thread owns
+constexpr int kPairs = kVec / 2;           // held as 16 packed float pairs (2i, 2i + 1)
 constexpr float kRoundMagic = 12582912.0f; // 1.5 * 2^23: x + magic rounds x to an integer (RNE)
 constexpr unsigned kFull = 0xffffffffu;
 
@@ -36,135 +39,244 @@ struct Norm {  // 1 / sqrt(G), exact
   static constexpr float value = G == 4 ? 0.5f : G == 16 ? 0.25f : G == 64 ? 0.125f : 0.0625f;
 };
 
-__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
-
-__device__ __forceinline__ void load_bf16_chunk(const uint16_t* p, float (&v)[kChunk]) {
-  const uint4* q = reinterpret_cast<const uint4*>(p);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const uint4 u = __ldg(q + i);
-    v[8 * i + 0] = bf16_lo(u.x);
-    v[8 * i + 1] = bf16_hi(u.x);
-    v[8 * i + 2] = bf16_lo(u.y);
-    v[8 * i + 3] = bf16_hi(u.y);
-    v[8 * i + 4] = bf16_lo(u.z);
-    v[8 * i + 5] = bf16_hi(u.z);
-    v[8 * i + 6] = bf16_lo(u.w);
-    v[8 * i + 7] = bf16_hi(u.w);
-  }
+// ---------------------------------------------------------------- packed pairs
+// sm_100 executes two float32 operations per instruction on a 64-bit register
+// pair; the butterflies, the scaling and the code rounding use these forms.
+__device__ __forceinline__ uint64_t pk(float lo, float hi) {
+  return (static_cast<uint64_t>(__float_as_uint(hi)) << 32) | __float_as_uint(lo);
+}
+__device__ __forceinline__ float plo(uint64_t p) { return __uint_as_float(static_cast<uint32_t>(p)); }
+__device__ __forceinline__ float phi(uint64_t p) { return __uint_as_float(static_cast<uint32_t>(p >> 32)); }
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t mulrz2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rz.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
 }
 
-__device__ __forceinline__ void load_i8_chunk(const int8_t* p, float (&v)[kChunk]) {
-  const int4* q = reinterpret_cast<const int4*>(p);
+// ---------------------------------------------------------------- shared memory
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void sts128(uint32_t addr, uint64_t a, uint64_t b) {
+  asm volatile("st.shared.v2.b64 [%0], {%1, %2};" ::"r"(addr), "l"(a), "l"(b) : "memory");
+}
+__device__ __forceinline__ void lds128(uint32_t addr, uint64_t& a, uint64_t& b) {
+  asm volatile("ld.shared.v2.b64 {%0, %1}, [%2];" : "=l"(a), "=l"(b) : "r"(addr) : "memory");
+}
+
+// ---------------------------------------------------------------- loads
+// 32 bf16 at p (16-byte aligned) -> P[i] = (p[2i], p[2i + 1]).
+__device__ __forceinline__ void load_bf16_32(const uint16_t* p, uint64_t (&P)[kPairs]) {
+  const uint4* q = reinterpret_cast<const uint4*>(p);
+  uint4 u[4];
 #pragma unroll
-  for (int i = 0; i < 2; ++i) {
-    const int4 u = __ldg(q + i);
-    const int w[4] = {u.x, u.y, u.z, u.w};
+  for (int j = 0; j < 4; ++j) u[j] = __ldg(q + j);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t w[4] = {u[j].x, u[j].y, u[j].z, u[j].w};
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-#pragma unroll
-      for (int b = 0; b < 4; ++b) {
-        v[16 * i + 4 * k + b] = static_cast<float>(static_cast<int8_t>((w[k] >> (8 * b)) & 0xff));
-      }
+      P[4 * j + k] = pk(__uint_as_float(w[k] << 16), __uint_as_float(w[k] & 0xffff0000u));
     }
   }
 }
 
-// Butterfly stages whose partner lies in the same chunk (stride < min(G, 32)).
+// 32 int8 at p (16-byte aligned) -> P[i] = (p[2i], p[2i + 1]).
+__device__ __forceinline__ void load_i8_32(const int8_t* p, uint64_t (&P)[kPairs]) {
+  const int4* q = reinterpret_cast<const int4*>(p);
+  int4 u[2];
+#pragma unroll
+  for (int j = 0; j < 2; ++j) u[j] = __ldg(q + j);
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    const int w[4] = {u[j].x, u[j].y, u[j].z, u[j].w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      P[8 * j + 2 * k] = pk(static_cast<float>(static_cast<int8_t>(w[k])),
+                            static_cast<float>(static_cast<int8_t>(w[k] >> 8)));
+      P[8 * j + 2 * k + 1] = pk(static_cast<float>(static_cast<int8_t>(w[k] >> 16)),
+                                static_cast<float>(w[k] >> 24));
+    }
+  }
+}
+
+// ---------------------------------------------------------------- butterflies
+// Unnormalised Walsh-Hadamard transform of every G-group, y = x . H_G, for the
+// 32-element chunk of each lane (pairs P[i] = elements (2i, 2i + 1)).
+//   bit 0: the two halves of each pair;   bits 1..4: across pairs (packed);
+//   G == 64: bit 5 across lanes l and l ^ 1 (warp shuffle);
+//   G == 256: bits 5..7 after one exchange through shared memory: the 8 lanes
+//   of a group each write their 32 elements as 8 slots of 16 bytes and read
+//   slot t (elements 4t .. 4t + 3) of every lane of the group; slot m of lane
+//   s sits at 8 s + (m ^ s), so the 8 lanes of a quarter-warp (one group) hit
+//   8 distinct bank quads on both sides.  Afterwards lane t holds in
+//   P[2 s + q] the elements (32 s + 4t + 2q, 32 s + 4t + 2q + 1), s = 0..7.
+constexpr int kXchBytesPerWarp = 4 * 64 * 16;  // 4 groups x 64 slots
+
 template <int G>
-__device__ __forceinline__ void fwht_in_chunk(float (&v)[kChunk]) {
-  constexpr int kTop = G < kChunk ? G : kChunk;
+__device__ __forceinline__ void fwht32(uint64_t (&P)[kPairs], uint32_t xch, uint32_t lane) {
+#pragma unroll
+  for (int i = 0; i < kPairs; ++i) {  // bit 0
+    const float a = plo(P[i]), b = phi(P[i]);
+    P[i] = pk(a + b, a - b);
+  }
+  constexpr int kTop = (G < kVec ? G : kVec) / 2;  // pair-index stages (bits 1..)
 #pragma unroll
   for (int h = 1; h < kTop; h <<= 1) {
 #pragma unroll
-    for (int i = 0; i < kChunk; ++i) {
+    for (int i = 0; i < kPairs; ++i) {
       if ((i & h) == 0) {
-        const float a = v[i], b = v[i + h];
-        v[i] = a + b;
-        v[i + h] = a - b;
+        const uint64_t a = P[i], b = P[i + h];
+        P[i] = add2(a, b);
+        P[i + h] = sub2(a, b);
+      }
+    }
+  }
+  if constexpr (G == 64) {
+    const float sg = (lane & 1) ? -1.f : 1.f;  // the upper lane keeps a - b
+    const uint64_t sgn = pk(sg, sg);
+#pragma unroll
+    for (int i = 0; i < kPairs; ++i) {
+      const float lo = __shfl_xor_sync(kFull, plo(P[i]), 1);
+      const float hi = __shfl_xor_sync(kFull, phi(P[i]), 1);
+      P[i] = fma2(sgn, P[i], pk(lo, hi));
+    }
+  }
+  if constexpr (G == 256) {
+    const uint32_t t = lane & 7;
+    const uint32_t g = xch + (lane >> 3) * (64 * 16);
+#pragma unroll
+    for (int m = 0; m < 8; ++m) sts128(g + 16 * (8 * t + (m ^ t)), P[2 * m], P[2 * m + 1]);
+    __syncwarp();
+#pragma unroll
+    for (int s = 0; s < 8; ++s) lds128(g + 16 * (8 * s + (t ^ s)), P[2 * s], P[2 * s + 1]);
+    __syncwarp();
+#pragma unroll
+    for (int h = 1; h < 8; h <<= 1) {  // bits 5..7: across source lanes
+#pragma unroll
+      for (int s = 0; s < 8; ++s) {
+        if ((s & h) == 0) {
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            const uint64_t a = P[2 * s + q], b = P[2 * (s + h) + q];
+            P[2 * s + q] = add2(a, b);
+            P[2 * (s + h) + q] = sub2(a, b);
+          }
+        }
       }
     }
   }
 }
 
-// Butterfly stages across the G/32 lanes that hold one group (G > 32).  Every
-// lane of the warp must execute this (full-mask shuffles).
-template <int G>
-__device__ __forceinline__ void fwht_across_lanes(float (&v)[kChunk], uint32_t lane) {
-#pragma unroll
-  for (int m = 1; m < G / kChunk; m <<= 1) {
-    const float sgn = (lane & m) ? -1.f : 1.f;  // upper partner keeps a - b
-#pragma unroll
-    for (int i = 0; i < kChunk; ++i) {
-      const float p = __shfl_xor_sync(kFull, v[i], m);
-      v[i] = fmaf(sgn, v[i], p);
-    }
-  }
-}
-
-template <int G>
-__device__ __forceinline__ void fwht_chunk(float (&v)[kChunk], uint32_t lane) {
-  fwht_in_chunk<G>(v);
-  if constexpr (G > kChunk) fwht_across_lanes<G>(v, lane);
-}
-
-// Code of v * mul rounded half to even; |v * mul| <= 127.5 is required.
-// Returns the code in the low byte (two's complement) of a 32-bit word.
-__device__ __forceinline__ uint32_t round_code(float v, float mul) {
-  return __float_as_uint(fmaf(v, mul, kRoundMagic));
-}
-
+// ---------------------------------------------------------------- outputs
 __device__ __forceinline__ uint32_t pack4(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
 }
 
-// 32 codes of one chunk -> 32 bytes at dst (16-byte aligned).
-__device__ __forceinline__ void store_codes(int8_t* dst, const float (&v)[kChunk], float mul) {
+// Writes the low byte of each half of R (a code in two's complement) where
+// fwht32 left that element; `base` = first element of the lane's chunk.
+template <int G>
+__device__ __forceinline__ void store_code_bytes(int8_t* base, const uint64_t (&R)[kPairs],
+                                                 uint32_t lane) {
   uint32_t w[8];
 #pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    w[k] = pack4(round_code(v[4 * k], mul), round_code(v[4 * k + 1], mul),
-                 round_code(v[4 * k + 2], mul), round_code(v[4 * k + 3], mul));
+  for (int j = 0; j < 8; ++j) {
+    w[j] = pack4(static_cast<uint32_t>(R[2 * j]), static_cast<uint32_t>(R[2 * j] >> 32),
+                 static_cast<uint32_t>(R[2 * j + 1]), static_cast<uint32_t>(R[2 * j + 1] >> 32));
   }
-  uint4* q = reinterpret_cast<uint4*>(dst);
-  q[0] = make_uint4(w[0], w[1], w[2], w[3]);
-  q[1] = make_uint4(w[4], w[5], w[6], w[7]);
-}
-
-// Slow but exact-division codes, for scales so small that 1/s overflows.
-__device__ __forceinline__ void store_codes_div(int8_t* dst, const float (&v)[kChunk], float norm,
-                                                float s) {
-  uint32_t w[8];
+  if constexpr (G == 256) {
+    const uint32_t t = lane & 7;
+    int8_t* grp = base - kVec * t;
 #pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    uint32_t c[4];
-#pragma unroll
-    for (int b = 0; b < 4; ++b) {
-      float q = rintf(__fdiv_rn(v[4 * k + b] * norm, s));
-      q = fminf(fmaxf(q, -127.f), 127.f);
-      c[b] = static_cast<uint32_t>(static_cast<int32_t>(q));
-    }
-    w[k] = pack4(c[0], c[1], c[2], c[3]);
+    for (int s = 0; s < 8; ++s) *reinterpret_cast<uint32_t*>(grp + 32 * s + 4 * t) = w[s];
+  } else {
+    uint4* q = reinterpret_cast<uint4*>(base);
+    q[0] = make_uint4(w[0], w[1], w[2], w[3]);
+    q[1] = make_uint4(w[4], w[5], w[6], w[7]);
   }
-  uint4* q = reinterpret_cast<uint4*>(dst);
-  q[0] = make_uint4(w[0], w[1], w[2], w[3]);
-  q[1] = make_uint4(w[4], w[5], w[6], w[7]);
 }
 
-// bf16 bits of the exact product s * v rounded once to nearest-even.  The
-// product is first rounded toward zero to float32 with the last bit forced to
-// one when inexact ("round to odd"); rounding that to the 8-bit bf16 mantissa
-// is then the correctly rounded result (float32 keeps >= 2 extra bits).
-__device__ __forceinline__ float round_to_odd_product(float s, float v) {
-  const float p = __fmul_rz(s, v);
-  const float e = __fmaf_rn(s, v, -p);  // exact remainder
-  return __uint_as_float(__float_as_uint(p) | (e != 0.f ? 1u : 0u));
+// Codes rne(v * mul) of the 32 values (|v * mul| <= 127.5): one packed FMA
+// against 1.5 * 2^23 leaves each code in the low byte of its float.
+template <int G>
+__device__ __forceinline__ void store_codes32(int8_t* base, const uint64_t (&P)[kPairs], float mul,
+                                             uint32_t lane) {
+  const uint64_t m2 = pk(mul, mul), magic2 = pk(kRoundMagic, kRoundMagic);
+  uint64_t R[kPairs];
+#pragma unroll
+  for (int i = 0; i < kPairs; ++i) R[i] = fma2(P[i], m2, magic2);
+  store_code_bytes<G>(base, R, lane);
 }
 
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-  const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+// Exact-division codes rne(v * norm / s), for scales so small that 1/s overflows.
+template <int G>
+__device__ __forceinline__ void store_codes32_div(int8_t* base, const uint64_t (&P)[kPairs],
+                                                  float norm, float s, uint32_t lane) {
+  uint64_t R[kPairs];
+#pragma unroll
+  for (int i = 0; i < kPairs; ++i) {
+    const float a = fminf(fmaxf(rintf(__fdiv_rn(plo(P[i]) * norm, s)), -127.f), 127.f);
+    const float b = fminf(fmaxf(rintf(__fdiv_rn(phi(P[i]) * norm, s)), -127.f), 127.f);
+    R[i] = pk(a + kRoundMagic, b + kRoundMagic);
+  }
+  store_code_bytes<G>(base, R, lane);
+}
+
+// bf16 pair of the exact products s * v, each rounded once to nearest-even:
+// the product is rounded toward zero to float32 and its last bit forced to one
+// when inexact ("round to odd"); float32 keeps more than two extra bits, so
+// rounding that to bf16 is the correctly rounded result.
+__device__ __forceinline__ uint32_t bf16x2_exact_product(uint64_t s2, uint64_t v) {
+  const uint64_t p = mulrz2(s2, v);
+  const uint64_t e = fma2(s2, v, p ^ 0x8000000080000000ull);  // exact remainder s*v - p
+  uint32_t lo = static_cast<uint32_t>(p), hi = static_cast<uint32_t>(p >> 32);
+  lo |= (static_cast<uint32_t>(e) << 1) != 0u ? 1u : 0u;
+  hi |= (static_cast<uint32_t>(e >> 32) << 1) != 0u ? 1u : 0u;
+  const __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(lo), __uint_as_float(hi));
   return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+template <int G>
+__device__ __forceinline__ void store_bf16_32(uint16_t* base, const uint64_t (&P)[kPairs], float sn,
+                                              uint32_t lane) {
+  const uint64_t s2 = pk(sn, sn);
+  uint32_t w[kPairs];
+#pragma unroll
+  for (int i = 0; i < kPairs; ++i) w[i] = bf16x2_exact_product(s2, P[i]);  // elements 2i, 2i + 1
+  if constexpr (G == 256) {
+    const uint32_t t = lane & 7;
+    uint16_t* grp = base - kVec * t;
+#pragma unroll
+    for (int s = 0; s < 8; ++s) {
+      *reinterpret_cast<uint2*>(grp + 32 * s + 4 * t) = make_uint2(w[2 * s], w[2 * s + 1]);
+    }
+  } else {
+    uint4* q = reinterpret_cast<uint4*>(base);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) q[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+  }
+}
+
+__device__ __forceinline__ float absmax32(const uint64_t (&P)[kPairs]) {
+  float m = 0.f;
+#pragma unroll
+  for (int i = 0; i < kPairs; ++i) m = fmaxf(m, fmaxf(fabsf(plo(P[i])), fabsf(phi(P[i]))));
+  return m;
 }
 
 __device__ __forceinline__ float warp_max(float a) {
@@ -173,76 +285,64 @@ __device__ __forceinline__ float warp_max(float a) {
   return a;
 }
 
+template <int G>
+__host__ __device__ constexpr int xch_bytes_per_warp() {
+  return G == 256 ? kXchBytesPerWarp : 0;
+}
+
 // ===========================================================================
-// Sylvester path, activations: one team of `team_warps` warps per token.
-// The token's rotated row stays in registers between the absmax and the pack.
+// Sylvester path, activations: a team of `team_warps` warps per token, one
+// 32-element chunk per lane, all loads issued before any arithmetic.  The
+// token's rotated row stays in registers between the absmax and the pack.
 // ===========================================================================
-template <int G, int MAXC>
+template <int G>
 __global__ void __launch_bounds__(1024) rotate_quant_act_hadamard(
     const uint16_t* __restrict__ x, int64_t M, int K, int team_warps, int rows_per_cta,
     int8_t* __restrict__ xq, float* __restrict__ s_tok) {
+  extern __shared__ __align__(16) uint8_t xch_all[];
   __shared__ float red[32];
   const int warp = threadIdx.x >> 5;
   const uint32_t lane = threadIdx.x & 31;
   const int team = warp / team_warps;
-  const int tpr = team_warps * 32;
-  const int t = (warp % team_warps) * 32 + lane;
+  const int t = (warp % team_warps) * 32 + static_cast<int>(lane);  // chunk within the token
   const int64_t row = static_cast<int64_t>(blockIdx.x) * rows_per_cta + team;
   const bool row_ok = row < M;  // uniform over the team
-  const int nch = K / kChunk;
-  const uint16_t* xr = x + row * K;
+  const int nch = K / kVec;
+  const bool ok = row_ok && t < nch;  // whole groups agree (K % G == 0)
+  const uint32_t xch = smem_addr(xch_all) + warp * xch_bytes_per_warp<G>();
 
-  float v[MAXC][kChunk];
+  uint64_t P[kPairs];
+  if (ok) {
+    load_bf16_32(x + row * K + static_cast<int64_t>(t) * kVec, P);
+  } else {
 #pragma unroll
-  for (int j = 0; j < MAXC; ++j) {
-    const int c = j * tpr + t;
-    if (row_ok && c < nch) {
-      load_bf16_chunk(xr + static_cast<int64_t>(c) * kChunk, v[j]);
-    } else {
-#pragma unroll
-      for (int i = 0; i < kChunk; ++i) v[j][i] = 0.f;
-    }
+    for (int i = 0; i < kPairs; ++i) P[i] = 0;
   }
-  float amax = 0.f;
-#pragma unroll
-  for (int j = 0; j < MAXC; ++j) {
-    fwht_chunk<G>(v[j], lane);
-#pragma unroll
-    for (int i = 0; i < kChunk; ++i) amax = fmaxf(amax, fabsf(v[j][i]));
-  }
-  amax = warp_max(amax);
+  fwht32<G>(P, xch, lane);
+  float amax = warp_max(absmax32(P));
   if (team_warps > 1) {
     if (lane == 0) red[warp] = amax;
     __syncthreads();
     amax = 0.f;
     for (int k = 0; k < team_warps; ++k) amax = fmaxf(amax, red[team * team_warps + k]);
   }
-  if (!row_ok) return;
+  if (!ok) return;
 
   constexpr float norm = Norm<G>::value;
   const float s = (amax * norm) / 127.f;  // s_tok = max |x_rot| / 127
   if (t == 0) s_tok[row] = s;
-  const float inv = s > 0.f ? 1.f / s : 0.f;
-  const float mul = norm * inv;  // exact: norm is a power of two
-  int8_t* qr = xq + row * K;
+  const float mul = norm * (s > 0.f ? 1.f / s : 0.f);  // exact scaling: norm is a power of two
+  int8_t* dst = xq + row * K + static_cast<int64_t>(t) * kVec;
   if (mul <= 3.0e38f) {
-#pragma unroll
-    for (int j = 0; j < MAXC; ++j) {
-      const int c = j * tpr + t;
-      if (c < nch) store_codes(qr + static_cast<int64_t>(c) * kChunk, v[j], mul);
-    }
+    store_codes32<G>(dst, P, mul, lane);
   } else {
-#pragma unroll
-    for (int j = 0; j < MAXC; ++j) {
-      const int c = j * tpr + t;
-      if (c < nch) store_codes_div(qr + static_cast<int64_t>(c) * kChunk, v[j], norm, s);
-    }
+    store_codes32_div<G>(dst, P, norm, s, lane);
   }
 }
 
 // ===========================================================================
-// Sylvester path over a flat [rows, K] tensor, one chunk per thread per step.
-// Groups never straddle rows (K % G == 0, K % 32 == 0).
+// Sylvester path over a flat [rows, K] tensor, one 32-element chunk per
+// thread.  Groups never straddle rows (K % G == 0, K % 32 == 0).
 // ===========================================================================
 enum FlatMode { kFlatAbsmax = 0, kFlatQuant = 1, kFlatDequant = 2 };
 
@@ -252,58 +352,29 @@ __global__ void __launch_bounds__(256) hadamard_flat(const void* __restrict__ in
                                                      const float* __restrict__ scale,
                                                      void* __restrict__ out,
                                                      unsigned int* __restrict__ absmax_bits) {
+  extern __shared__ __align__(16) uint8_t xch_all[];
   const uint32_t lane = threadIdx.x & 31;
-  const int64_t warp_global = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int64_t warp_stride = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  const int64_t c = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const bool ok = c < nchunks;  // whole groups agree: nchunks % (G / 32) == 0
+  const uint32_t xch = smem_addr(xch_all) + (threadIdx.x >> 5) * xch_bytes_per_warp<G>();
   constexpr float norm = Norm<G>::value;
-  float amax = 0.f;
-  float mul = 0.f;
-  if constexpr (MODE == kFlatQuant) {
-    const float a = __uint_as_float(*absmax_bits);
-    const float s = a / 127.f;
-    mul = s > 0.f ? norm * (1.f / s) : 0.f;
-  }
-  for (int64_t base = warp_global * 32; base < nchunks; base += warp_stride * 32) {
-    const int64_t c = base + lane;
-    const bool ok = c < nchunks;
-    float v[kChunk];
-    if (ok) {
-      if constexpr (MODE == kFlatDequant) {
-        load_i8_chunk(static_cast<const int8_t*>(in) + c * kChunk, v);
-      } else {
-        load_bf16_chunk(static_cast<const uint16_t*>(in) + c * kChunk, v);
-      }
+
+  uint64_t P[kPairs];
+  if (ok) {
+    if constexpr (MODE == kFlatDequant) {
+      load_i8_32(static_cast<const int8_t*>(in) + c * kVec, P);
     } else {
-#pragma unroll
-      for (int i = 0; i < kChunk; ++i) v[i] = 0.f;
+      load_bf16_32(static_cast<const uint16_t*>(in) + c * kVec, P);
     }
-    fwht_chunk<G>(v, lane);
-    if constexpr (MODE == kFlatAbsmax) {
+  } else {
 #pragma unroll
-      for (int i = 0; i < kChunk; ++i) amax = fmaxf(amax, fabsf(v[i]));
-    } else if constexpr (MODE == kFlatQuant) {
-      if (ok) store_codes(static_cast<int8_t*>(out) + c * kChunk, v, mul);
-    } else {
-      if (ok) {
-        const float sw = PER_ROW_SCALE ? scale[c / chunks_per_row] : scale[0];
-        const float sn = sw * norm;  // exact
-        uint32_t w[16];
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          w[k] = pack_bf16x2(round_to_odd_product(sn, v[2 * k]),
-                             round_to_odd_product(sn, v[2 * k + 1]));
-        }
-        uint4* q = reinterpret_cast<uint4*>(static_cast<uint16_t*>(out) + c * kChunk);
-        q[0] = make_uint4(w[0], w[1], w[2], w[3]);
-        q[1] = make_uint4(w[4], w[5], w[6], w[7]);
-        q[2] = make_uint4(w[8], w[9], w[10], w[11]);
-        q[3] = make_uint4(w[12], w[13], w[14], w[15]);
-      }
-    }
+    for (int i = 0; i < kPairs; ++i) P[i] = 0;
   }
+  fwht32<G>(P, xch, lane);
+
   if constexpr (MODE == kFlatAbsmax) {
     __shared__ float red[8];
-    amax = warp_max(amax);
+    const float amax = warp_max(absmax32(P));
     if (lane == 0) red[threadIdx.x >> 5] = amax;
     __syncthreads();
     if (threadIdx.x == 0) {
@@ -311,6 +382,21 @@ __global__ void __launch_bounds__(256) hadamard_flat(const void* __restrict__ in
       for (int k = 0; k < static_cast<int>(blockDim.x >> 5); ++k) m = fmaxf(m, red[k]);
       atomicMax(absmax_bits, __float_as_uint(m * norm));  // non-negative: bit order = value order
     }
+  } else if constexpr (MODE == kFlatQuant) {
+    if (!ok) return;
+    const float a = __uint_as_float(*absmax_bits);
+    const float s = a / 127.f;
+    const float mul = s > 0.f ? norm * (1.f / s) : 0.f;
+    int8_t* dst = static_cast<int8_t*>(out) + c * kVec;
+    if (mul <= 3.0e38f) {
+      store_codes32<G>(dst, P, mul, lane);
+    } else {
+      store_codes32_div<G>(dst, P, norm, s, lane);
+    }
+  } else {
+    if (!ok) return;
+    const float sw = PER_ROW_SCALE ? scale[c / chunks_per_row] : scale[0];
+    store_bf16_32<G>(static_cast<uint16_t*>(out) + c * kVec, P, sw * norm, lane);
   }
 }
 
@@ -434,19 +520,41 @@ __global__ void finalize_scales(float* __restrict__ s, int64_t n) {
   if (i < n) s[i] = s[i] / 127.f;
 }
 
+template <typename Kern>
+cudaError_t allow_smem(Kern kern, size_t bytes) {
+  if (bytes <= 48 * 1024) return cudaSuccess;
+  return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              static_cast<int>(bytes));
+}
+
 template <int G>
 cudaError_t rqa_hadamard(const uint16_t* x, int64_t M, int64_t K, int8_t* xq, float* s_tok,
                          cudaStream_t stream) {
   // A token's row is held by a team of ceil(K / 1024) warps, one 32-element
-  // chunk per lane (64 registers), so many teams stay resident per SM and the
-  // load, butterfly and store phases of different teams overlap.
-  const int nch = static_cast<int>(K / kChunk);
+  // chunk per lane; small rows share a CTA (8 warps).
+  const int nch = static_cast<int>(K / kVec);
   const int team_warps = (nch + 31) / 32;
   const int rows_per_cta = team_warps >= 8 ? 1 : 8 / team_warps;
+  const int warps = team_warps * rows_per_cta;
+  const size_t smem = static_cast<size_t>(warps) * xch_bytes_per_warp<G>();
+  cudaError_t e = allow_smem(rotate_quant_act_hadamard<G>, smem);
+  if (e != cudaSuccess) return e;
   const int64_t grid = (M + rows_per_cta - 1) / rows_per_cta;
-  rotate_quant_act_hadamard<G, 1><<<static_cast<unsigned>(grid), 32 * team_warps * rows_per_cta,
-                                    0, stream>>>(x, M, static_cast<int>(K), team_warps,
-                                                 rows_per_cta, xq, s_tok);
+  rotate_quant_act_hadamard<G><<<static_cast<unsigned>(grid), 32 * warps, smem, stream>>>(
+      x, M, static_cast<int>(K), team_warps, rows_per_cta, xq, s_tok);
+  return cudaGetLastError();
+}
+
+template <int G, int MODE, bool PER_ROW>
+cudaError_t flat_launch(const void* in, int64_t nchunks, int64_t chunks_per_row,
+                        const float* scale, void* out, unsigned int* absmax_bits,
+                        cudaStream_t stream) {
+  constexpr int kThreadsFlat = 256;
+  const size_t smem = (kThreadsFlat / 32) * xch_bytes_per_warp<G>();
+  int64_t grid = (nchunks + kThreadsFlat - 1) / kThreadsFlat;  // one chunk per thread
+  if (grid < 1) grid = 1;
+  hadamard_flat<G, MODE, PER_ROW><<<static_cast<unsigned>(grid), kThreadsFlat, smem, stream>>>(
+      in, nchunks, chunks_per_row, scale, out, absmax_bits);
   return cudaGetLastError();
 }
 
@@ -464,18 +572,6 @@ cudaError_t dense_launch(const TIn* in, int64_t group_rows, int64_t groups_per_t
   const int64_t grid = (group_rows + TMR - 1) / TMR;
   kern<<<static_cast<unsigned>(grid), 256, smem, stream>>>(in, group_rows, groups_per_token, Rm,
                                                            scale, scale_len, out, absmax_bits);
-  return cudaGetLastError();
-}
-
-template <int G, int MODE, bool PER_ROW>
-cudaError_t flat_launch(const void* in, int64_t nchunks, int64_t chunks_per_row,
-                        const float* scale, void* out, unsigned int* absmax_bits,
-                        cudaStream_t stream) {
-  const int64_t warps = (nchunks + 31) / 32;
-  int64_t grid = (warps + 7) / 8;  // one chunk per thread
-  if (grid < 1) grid = 1;
-  hadamard_flat<G, MODE, PER_ROW><<<static_cast<unsigned>(grid), 256, 0, stream>>>(
-      in, nchunks, chunks_per_row, scale, out, absmax_bits);
   return cudaGetLastError();
 }
 
@@ -521,14 +617,14 @@ cudaError_t launch_dequant_derotate(const convrot_rotation_s* R, const int8_t* W
                                     const float* s_w, int64_t s_w_len, int64_t N, int64_t K,
                                     uint16_t* W_hat, cudaStream_t stream) {
   if (R->is_sylvester) {
-    const int64_t nchunks = N * K / kChunk;
+    const int64_t nchunks = N * K / kVec;
     return by_group_size(R->G, [&](auto g) {
       constexpr int Gv = decltype(g)::value;
       if (s_w_len == 1) {
-        return flat_launch<Gv, kFlatDequant, false>(Wq, nchunks, K / kChunk, s_w, W_hat, nullptr,
+        return flat_launch<Gv, kFlatDequant, false>(Wq, nchunks, K / kVec, s_w, W_hat, nullptr,
                                                     stream);
       }
-      return flat_launch<Gv, kFlatDequant, true>(Wq, nchunks, K / kChunk, s_w, W_hat, nullptr,
+      return flat_launch<Gv, kFlatDequant, true>(Wq, nchunks, K / kVec, s_w, W_hat, nullptr,
                                                  stream);
     });
   }
@@ -545,14 +641,13 @@ cudaError_t launch_quantize_weight(const convrot_rotation_s* R, const uint16_t* 
   cudaError_t e = cudaMemsetAsync(amax, 0, sizeof(float), stream);
   if (e != cudaSuccess) return e;
   if (R->is_sylvester) {
-    const int64_t nchunks = N * K / kChunk;
+    const int64_t nchunks = N * K / kVec;
     e = by_group_size(R->G, [&](auto g) {
       constexpr int Gv = decltype(g)::value;
-      cudaError_t r = flat_launch<Gv, kFlatAbsmax, false>(W, nchunks, K / kChunk, nullptr,
-                                                          nullptr, amax, stream);
+      cudaError_t r = flat_launch<Gv, kFlatAbsmax, false>(W, nchunks, K / kVec, nullptr, nullptr,
+                                                          amax, stream);
       if (r != cudaSuccess) return r;
-      return flat_launch<Gv, kFlatQuant, false>(W, nchunks, K / kChunk, nullptr, Wq, amax,
-                                                stream);
+      return flat_launch<Gv, kFlatQuant, false>(W, nchunks, K / kVec, nullptr, Wq, amax, stream);
     });
   } else {
     const int64_t gpt = K / R->G;
