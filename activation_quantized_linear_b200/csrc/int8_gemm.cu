@@ -5,16 +5,21 @@
 //   acc[m, n] = sum_k xq[m, k] * Wq[n, k]                       (exact int32)
 //   y[m, n]   = bf16_rn(float(acc) * (s_tok[m] * s_w[n|0]) + bias[n])
 //
-// Structure (one CTA per SM, persistent over 128 x 256 output tiles):
-//   warp 0      TMA producer: 128 x 128 A and 256 x 128 B int8 tiles, 128-byte
-//               swizzle, into a 4-stage shared-memory ring (48 KB per stage);
-//   warp 1      allocates 512 TMEM columns, one thread issues
-//               tcgen05.mma.cta_group::1.kind::i8 (M=128, N=256, K=32) into one
-//               of two 256-column int32 accumulators, tcgen05.commit frees the
-//               stage / publishes the accumulator;
+// Structure (persistent; one CTA per SM):
+//   warp 0      TMA producer: A and B int8 tiles of 128-byte rows, 128-byte
+//               swizzle, into a shared-memory ring;
+//   warp 1      allocates 512 TMEM columns; one thread issues tcgen05.mma
+//               kind::i8 (K = 32 per instruction) into one of two 256-column
+//               int32 accumulators; tcgen05.commit frees the stage / publishes
+//               the accumulator;
 //   warps 2..5  epilogue: tcgen05.ld 32 columns at a time, rescale, bias, bf16,
 //               128-bit global stores; then release the accumulator so the MMA
 //               of the next tile overlaps this tile's epilogue.
+// For more than 128 tokens, CTA pairs (clusters of two SMs, cta_group::2) work
+// on 256 x 256 tiles: each CTA loads its 128 rows of A and 128 rows of B (no
+// multicast), the even CTA issues M=256 x N=256 MMAs whose accumulators are
+// split across the two CTAs' TMEM, and commits signal both CTAs' barriers.  A
+// pair moves 2/3 of the operand bytes per MMA that two single CTAs would.
 // Every mbarrier wait is bounded by the global timer.  A wait that runs out
 // records CONVROT_ERR_TIMEOUT in the device status word; the CTA then stops
 // issuing work, drains what it issued and frees its TMEM before returning.
@@ -29,24 +34,37 @@
 #include "sm100_ptx.cuh"
 
 namespace convrot {
-
 namespace {
 
-constexpr int BM = 128;
-constexpr int BN = 256;
-constexpr int BK = 128;  // bytes = int8 elements; one 128-byte swizzle row
+constexpr int BM = 128;       // accumulator rows per CTA (TMEM lanes)
+constexpr int BN = 256;       // accumulator columns per tile
+constexpr int BK = 128;       // bytes = int8 elements per stage; one 128-byte swizzle row
 constexpr int UMMA_K = 32;
-constexpr int STAGES = 4;
 constexpr int A_STAGE = BM * BK;
-constexpr int B_STAGE = BN * BK;
-constexpr int STAGE_BYTES = A_STAGE + B_STAGE;
-constexpr int ACC_COLS = BN;        // int32 accumulator columns per tile
+constexpr int ACC_COLS = BN;  // int32 accumulator columns per tile
 constexpr uint32_t TMEM_COLS = 2 * ACC_COLS;
 constexpr int kThreads = 192;
-constexpr int kEpiThreads = 128;
-constexpr int kGroupM = 8;          // tile raster: 8 M-tiles share a column sweep
+constexpr int kEpiWarps = 4;
+constexpr int kGroupM = 8;    // tile raster: 8 M-tiles share a column sweep
 constexpr uint64_t kWaitNs = 1000000000ull;  // 1 s per wait
-constexpr size_t kSmemBytes = 1024 /*align slack*/ + STAGES * STAGE_BYTES + 256 /*barriers*/;
+
+// Two variants share the kernel body:
+//   single: one CTA per tile of 128 x 256, B tile 256 x 128 per stage, 4 stages;
+//   pair:   a cluster of two CTAs per tile of 256 x 256 (cta_group::2); each CTA
+//           loads its 128 rows of A and its 128 rows of B per stage, 6 stages,
+//           and only the even CTA issues the MMAs.
+template <bool PAIR>
+struct Cfg {
+  static constexpr int kBRows = PAIR ? BN / 2 : BN;   // B rows loaded per CTA
+  static constexpr int kBStage = kBRows * BK;
+  static constexpr int kStageBytes = A_STAGE + kBStage;
+  static constexpr int kStages = PAIR ? 6 : 4;
+  static constexpr int kTileM = PAIR ? 2 * BM : BM;
+  static constexpr size_t kSmem = 1024 + kStages * kStageBytes + 256;
+  static constexpr uint32_t kIdesc = ptx::idesc_i8(kTileM, BN);
+  // bytes that complete one stage on the (leader's) full barrier
+  static constexpr uint32_t kTxBytes = (PAIR ? 2 : 1) * kStageBytes;
+};
 
 struct Params {
   const float* s_tok;
@@ -61,6 +79,7 @@ struct Params {
   unsigned int* status;  // device status word (bit 0: a wait ran out)
 };
 
+template <int STAGES>
 struct Barriers {
   uint64_t full[STAGES];
   uint64_t empty[STAGES];
@@ -81,13 +100,9 @@ __device__ __forceinline__ void tile_coords(int tile, int m_tiles, int n_tiles, 
   nb = local / gm;
 }
 
-__device__ __forceinline__ void record_timeout(Barriers* bars, unsigned int* status) {
+__device__ __forceinline__ void record_timeout(volatile uint32_t* abort_flag, unsigned int* status) {
   atomicOr(status, 1u);
-  *reinterpret_cast<volatile uint32_t*>(&bars->abort_flag) = 1u;
-}
-
-__device__ __forceinline__ bool aborted(Barriers* bars) {
-  return *reinterpret_cast<volatile uint32_t*>(&bars->abort_flag) != 0u;
+  *abort_flag = 1u;
 }
 
 __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity) {
@@ -131,27 +146,34 @@ __device__ __forceinline__ void store_s32_row32(int32_t* dst, const uint32_t (&r
   }
 }
 
+template <bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
     int8_gemm_tcgen05(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                       const Params p) {
+  using C = Cfg<PAIR>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* sA = smem;
-  uint8_t* sB = smem + STAGES * A_STAGE;
-  Barriers* bars = reinterpret_cast<Barriers*>(smem + STAGES * STAGE_BYTES);
+  uint8_t* sB = smem + C::kStages * A_STAGE;
+  auto* bars = reinterpret_cast<Barriers<C::kStages>*>(smem + C::kStages * C::kStageBytes);
+  volatile uint32_t* abort_flag = &bars->abort_flag;
 
   const int warp = threadIdx.x >> 5;
   const uint32_t lane = threadIdx.x & 31;
+  const uint32_t rank = PAIR ? ptx::cluster_ctarank() : 0;  // CTA within the pair
+  const bool leader = rank == 0;
+  const int unit = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int units = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
+    for (int s = 0; s < C::kStages; ++s) {
       ptx::mbar_init(&bars->full[s], 1);
       ptx::mbar_init(&bars->empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
       ptx::mbar_init(&bars->acc_full[a], 1);
-      ptx::mbar_init(&bars->acc_empty[a], kEpiThreads);
+      ptx::mbar_init(&bars->acc_empty[a], (PAIR ? 2 : 1) * kEpiWarps);
     }
     ptx::mbar_init(&bars->drain, 1);
     bars->abort_flag = 0;
@@ -160,14 +182,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::tma_prefetch_desc(&tmB);
   }
   if (warp == 1) {
-    ptx::tmem_alloc(&bars->tmem_base, TMEM_COLS);
-    ptx::tmem_relinquish();
+    if constexpr (PAIR) {
+      ptx::tmem_alloc_pair(&bars->tmem_base, TMEM_COLS);
+      ptx::tmem_relinquish_pair();
+    } else {
+      ptx::tmem_alloc(&bars->tmem_base, TMEM_COLS);
+      ptx::tmem_relinquish();
+    }
   }
   ptx::tc_fence_before();
-  __syncthreads();
+  if constexpr (PAIR) {
+    ptx::cluster_sync();  // both CTAs' barriers initialised before any cross-CTA signal
+  } else {
+    __syncthreads();
+  }
   ptx::tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
-
   const int num_tiles = p.m_tiles * p.n_tiles;
 
   if (threadIdx.x == 0) {
@@ -176,41 +206,48 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t phase = 0;
     int last_stage = -1;
     uint32_t last_phase = 0;
-    for (int tile = blockIdx.x; tile < num_tiles && !aborted(bars); tile += gridDim.x) {
+    for (int tile = unit; tile < num_tiles && !*abort_flag; tile += units) {
       int mb, nb;
       tile_coords(tile, p.m_tiles, p.n_tiles, mb, nb);
+      const int a_row = mb * C::kTileM + static_cast<int>(rank) * BM;
+      const int b_row = nb * BN + static_cast<int>(rank) * C::kBRows;
       for (int kb = 0; kb < p.num_kb; ++kb) {
         if (!wait_bounded(&bars->empty[stage], phase ^ 1u)) {
-          record_timeout(bars, p.status);
+          record_timeout(abort_flag, p.status);
           break;
         }
-        ptx::mbar_arrive_expect_tx(&bars->full[stage], STAGE_BYTES);
-        ptx::tma_load_2d(sA + stage * A_STAGE, &tmA, &bars->full[stage], kb * BK, mb * BM);
-        ptx::tma_load_2d(sB + stage * B_STAGE, &tmB, &bars->full[stage], kb * BK, nb * BN);
+        if constexpr (PAIR) {
+          if (leader) ptx::mbar_arrive_expect_tx(&bars->full[stage], C::kTxBytes);
+          ptx::tma_load_2d_pair(sA + stage * A_STAGE, &tmA, &bars->full[stage], kb * BK, a_row);
+          ptx::tma_load_2d_pair(sB + stage * C::kBStage, &tmB, &bars->full[stage], kb * BK, b_row);
+        } else {
+          ptx::mbar_arrive_expect_tx(&bars->full[stage], C::kTxBytes);
+          ptx::tma_load_2d(sA + stage * A_STAGE, &tmA, &bars->full[stage], kb * BK, a_row);
+          ptx::tma_load_2d(sB + stage * C::kBStage, &tmB, &bars->full[stage], kb * BK, b_row);
+        }
         last_stage = stage;
         last_phase = phase;
-        if (++stage == STAGES) {
+        if (++stage == C::kStages) {
           stage = 0;
           phase ^= 1u;
         }
       }
     }
-    if (aborted(bars) && last_stage >= 0) {
+    if (*abort_flag && last_stage >= 0 && leader) {
       // let the last copy land before the CTA's shared memory goes away
       ptx::mbar_wait(&bars->full[last_stage], last_phase, ptx::globaltimer_ns() + 10000000ull);
     }
-  } else if (threadIdx.x == 32) {
+  } else if (threadIdx.x == 32 && leader) {
     // ------------------------------------------------------------ MMA issuer
-    constexpr uint32_t idesc = ptx::idesc_i8(BM, BN);
     int stage = 0;
     uint32_t phase = 0;
     int local = 0;
     bool issued = false;
-    for (int tile = blockIdx.x; tile < num_tiles && !aborted(bars); tile += gridDim.x, ++local) {
+    for (int tile = unit; tile < num_tiles && !*abort_flag; tile += units, ++local) {
       const int acc = local & 1;
       const uint32_t acc_phase = (local >> 1) & 1;
       if (!wait_bounded(&bars->acc_empty[acc], acc_phase ^ 1u)) {
-        record_timeout(bars, p.status);
+        record_timeout(abort_flag, p.status);
         break;
       }
       ptx::tc_fence_after();
@@ -218,32 +255,48 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int kb = 0; kb < p.num_kb; ++kb) {
         if (!wait_bounded(&bars->full[stage], phase)) {
-          record_timeout(bars, p.status);
+          record_timeout(abort_flag, p.status);
           ok = false;
           break;
         }
         ptx::tc_fence_after();
         const uint32_t a_addr = ptx::smem_u32(sA + stage * A_STAGE);
-        const uint32_t b_addr = ptx::smem_u32(sB + stage * B_STAGE);
+        const uint32_t b_addr = ptx::smem_u32(sB + stage * C::kBStage);
 #pragma unroll
         for (int k = 0; k < BK / UMMA_K; ++k) {
           const uint64_t ad = ptx::smem_desc_k_sw128(a_addr + k * UMMA_K);
           const uint64_t bd = ptx::smem_desc_k_sw128(b_addr + k * UMMA_K);
-          ptx::mma_i8(d_tmem, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
+          if constexpr (PAIR) {
+            ptx::mma_i8_pair(d_tmem, ad, bd, C::kIdesc, (kb | k) != 0 ? 1u : 0u);
+          } else {
+            ptx::mma_i8(d_tmem, ad, bd, C::kIdesc, (kb | k) != 0 ? 1u : 0u);
+          }
         }
         issued = true;
-        ptx::mma_commit(&bars->empty[stage]);
-        if (++stage == STAGES) {
+        if constexpr (PAIR) {
+          ptx::mma_commit_pair(&bars->empty[stage]);
+        } else {
+          ptx::mma_commit(&bars->empty[stage]);
+        }
+        if (++stage == C::kStages) {
           stage = 0;
           phase ^= 1u;
         }
       }
       if (!ok) break;
-      ptx::mma_commit(&bars->acc_full[acc]);
+      if constexpr (PAIR) {
+        ptx::mma_commit_pair(&bars->acc_full[acc]);
+      } else {
+        ptx::mma_commit(&bars->acc_full[acc]);
+      }
     }
-    if (aborted(bars) && issued) {
+    if (*abort_flag && issued) {
       // every MMA issued so far must finish before TMEM is released
-      ptx::mma_commit(&bars->drain);
+      if constexpr (PAIR) {
+        ptx::mma_commit_pair_local(&bars->drain);
+      } else {
+        ptx::mma_commit(&bars->drain);
+      }
       ptx::mbar_wait(&bars->drain, 0, ptx::globaltimer_ns() + 10000000ull);
     }
   } else if (warp >= 2) {
@@ -251,18 +304,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int quarter = warp & 3;  // TMEM lanes this warp may read: 32*quarter ..
     const int row = quarter * 32 + static_cast<int>(lane);
     int local = 0;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
+    for (int tile = unit; tile < num_tiles; tile += units, ++local) {
       int mb, nb;
       tile_coords(tile, p.m_tiles, p.n_tiles, mb, nb);
       const int acc = local & 1;
       const uint32_t acc_phase = (local >> 1) & 1;
       const bool ready = __all_sync(0xffffffffu, wait_bounded(&bars->acc_full[acc], acc_phase));
       if (!ready) {
-        if (lane == 0) record_timeout(bars, p.status);
+        if (lane == 0) record_timeout(abort_flag, p.status);
         break;
       }
       ptx::tc_fence_after();
-      const int64_t m = static_cast<int64_t>(mb) * BM + row;
+      const int64_t m = static_cast<int64_t>(mb) * C::kTileM + rank * BM + row;
       const bool row_ok = m < p.M;
       float scale = 0.f;
       if (!p.out_s32 && row_ok) scale = p.s_tok[m] * (p.per_channel_scale ? 1.f : p.s_w[0]);
@@ -285,16 +338,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       ptx::tc_fence_before();
-      ptx::mbar_arrive(&bars->acc_empty[acc]);
+      __syncwarp();
+      if (lane == 0) {
+        if constexpr (PAIR) {
+          ptx::mbar_arrive_leader(&bars->acc_empty[acc]);
+        } else {
+          ptx::mbar_arrive(&bars->acc_empty[acc]);
+        }
+      }
     }
   }
 
   ptx::tc_fence_before();
-  __syncthreads();
+  if constexpr (PAIR) {
+    ptx::cluster_sync();  // the leader's MMAs into this CTA's TMEM are complete
+  } else {
+    __syncthreads();
+  }
   if (warp == 1) {
     __syncwarp();
     ptx::tc_fence_after();
-    ptx::tmem_dealloc(tmem, TMEM_COLS);
+    if constexpr (PAIR) {
+      ptx::tmem_dealloc_pair(tmem, TMEM_COLS);
+    } else {
+      ptx::tmem_dealloc(tmem, TMEM_COLS);
+    }
   }
 }
 
@@ -306,22 +374,42 @@ bool encode_operand(CUtensorMap* map, const int8_t* base, int64_t rows, int64_t 
                        static_cast<uint32_t>(box_rows));
 }
 
+template <bool PAIR>
+cudaError_t launch_variant(const GemmArgs& a, Params p, cudaStream_t stream) {
+  using C = Cfg<PAIR>;
+  CUtensorMap tmA, tmB;
+  if (!encode_operand(&tmA, a.A, a.M, a.K, BM) ||
+      !encode_operand(&tmB, a.B, a.N, a.K, C::kBRows)) {
+    return cudaErrorInvalidValue;
+  }
+  cudaError_t e = cudaFuncSetAttribute(int8_gemm_tcgen05<PAIR>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(C::kSmem));
+  if (e != cudaSuccess) return e;
+  p.m_tiles = static_cast<int>((a.M + C::kTileM - 1) / C::kTileM);
+  const int tiles = p.m_tiles * p.n_tiles;
+  const int per_unit = PAIR ? 2 : 1;
+  const int max_units = sm_count() / per_unit;
+  const int units = tiles < max_units ? tiles : max_units;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(units * per_unit));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = C::kSmem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = per_unit;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, int8_gemm_tcgen05<PAIR>, tmA, tmB, p);
+}
+
 }  // namespace
 
 cudaError_t launch_int8_gemm(const GemmArgs& a, cudaStream_t stream) {
   if (a.M == 0) return cudaSuccess;
-  CUtensorMap tmA, tmB;
-  if (!encode_operand(&tmA, a.A, a.M, a.K, BM) || !encode_operand(&tmB, a.B, a.N, a.K, BN)) {
-    return cudaErrorInvalidValue;
-  }
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(int8_gemm_tcgen05,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(kSmemBytes));
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
   Params p;
   cudaError_t se = status_word(&p.status);
   if (se != cudaSuccess) return se;
@@ -332,14 +420,12 @@ cudaError_t launch_int8_gemm(const GemmArgs& a, cudaStream_t stream) {
   p.M = a.M;
   p.N = a.N;
   p.num_kb = static_cast<int>((a.K + BK - 1) / BK);
-  p.m_tiles = static_cast<int>((a.M + BM - 1) / BM);
   p.n_tiles = static_cast<int>((a.N + BN - 1) / BN);
   p.per_channel_scale = a.s_w_len > 1 ? 1 : 0;
   p.out_s32 = a.out_s32 ? 1 : 0;
-  const int tiles = p.m_tiles * p.n_tiles;
-  const int grid = tiles < sm_count() ? tiles : sm_count();
-  int8_gemm_tcgen05<<<grid, kThreads, kSmemBytes, stream>>>(tmA, tmB, p);
-  return cudaGetLastError();
+  // CTA pairs (256-row tiles) once there is more than one 128-row block of tokens
+  if (a.M > BM) return launch_variant<true>(a, p, stream);
+  return launch_variant<false>(a, p, stream);
 }
 
 }  // namespace convrot
