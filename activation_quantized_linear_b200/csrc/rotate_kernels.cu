@@ -520,9 +520,11 @@ __global__ void finalize_scales(float* __restrict__ s, int64_t n) {
   if (i < n) s[i] = s[i] / 127.f;
 }
 
+// Opts the kernel in to `bytes` of dynamic shared memory (the default limit,
+// 48 KB, counts the kernel's static shared memory too).
 template <typename Kern>
 cudaError_t allow_smem(Kern kern, size_t bytes) {
-  if (bytes <= 48 * 1024) return cudaSuccess;
+  if (bytes == 0) return cudaSuccess;
   return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               static_cast<int>(bytes));
 }
@@ -551,6 +553,8 @@ cudaError_t flat_launch(const void* in, int64_t nchunks, int64_t chunks_per_row,
                         cudaStream_t stream) {
   constexpr int kThreadsFlat = 256;
   const size_t smem = (kThreadsFlat / 32) * xch_bytes_per_warp<G>();
+  cudaError_t e = allow_smem(hadamard_flat<G, MODE, PER_ROW>, smem);
+  if (e != cudaSuccess) return e;
   int64_t grid = (nchunks + kThreadsFlat - 1) / kThreadsFlat;  // one chunk per thread
   if (grid < 1) grid = 1;
   hadamard_flat<G, MODE, PER_ROW><<<static_cast<unsigned>(grid), kThreadsFlat, smem, stream>>>(
