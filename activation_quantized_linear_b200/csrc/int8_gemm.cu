@@ -45,7 +45,6 @@ constexpr int ACC_COLS = BN;  // int32 accumulator columns per tile
 constexpr uint32_t TMEM_COLS = 2 * ACC_COLS;
 constexpr int kThreads = 192;
 constexpr int kEpiWarps = 4;
-constexpr int kGroupM = 8;    // tile raster: 8 M-tiles share a column sweep
 constexpr uint64_t kWaitNs = 1000000000ull;  // 1 s per wait
 
 // Two variants share the kernel body:
@@ -74,6 +73,7 @@ struct Params {
   int64_t M, N;
   int num_kb;
   int m_tiles, n_tiles;
+  int group_m;
   int per_channel_scale;
   int out_s32;
   unsigned int* status;  // device status word (bit 0: a wait ran out)
@@ -90,11 +90,15 @@ struct Barriers {
   uint32_t abort_flag;
 };
 
-__device__ __forceinline__ void tile_coords(int tile, int m_tiles, int n_tiles, int& mb, int& nb) {
-  const int per_group = kGroupM * n_tiles;
+// Tile raster: groups of `group_m` M-tiles sweep all N-tiles, M fastest, so
+// the tiles in flight share their weight (B) tiles; with group_m = m_tiles
+// every weight tile is read once while all of A stays in L2.
+__device__ __forceinline__ void tile_coords(int tile, int m_tiles, int n_tiles, int group_m, int& mb,
+                                            int& nb) {
+  const int per_group = group_m * n_tiles;
   const int g = tile / per_group;
-  const int first_m = g * kGroupM;
-  const int gm = min(kGroupM, m_tiles - first_m);
+  const int first_m = g * group_m;
+  const int gm = min(group_m, m_tiles - first_m);
   const int local = tile - g * per_group;
   mb = first_m + local % gm;
   nb = local / gm;
@@ -208,7 +212,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t last_phase = 0;
     for (int tile = unit; tile < num_tiles && !*abort_flag; tile += units) {
       int mb, nb;
-      tile_coords(tile, p.m_tiles, p.n_tiles, mb, nb);
+      tile_coords(tile, p.m_tiles, p.n_tiles, p.group_m, mb, nb);
       const int a_row = mb * C::kTileM + static_cast<int>(rank) * BM;
       const int b_row = nb * BN + static_cast<int>(rank) * C::kBRows;
       for (int kb = 0; kb < p.num_kb; ++kb) {
@@ -306,7 +310,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int local = 0;
     for (int tile = unit; tile < num_tiles; tile += units, ++local) {
       int mb, nb;
-      tile_coords(tile, p.m_tiles, p.n_tiles, mb, nb);
+      tile_coords(tile, p.m_tiles, p.n_tiles, p.group_m, mb, nb);
       const int acc = local & 1;
       const uint32_t acc_phase = (local >> 1) & 1;
       const bool ready = __all_sync(0xffffffffu, wait_bounded(&bars->acc_full[acc], acc_phase));
@@ -387,6 +391,8 @@ cudaError_t launch_variant(const GemmArgs& a, Params p, cudaStream_t stream) {
                                        static_cast<int>(C::kSmem));
   if (e != cudaSuccess) return e;
   p.m_tiles = static_cast<int>((a.M + C::kTileM - 1) / C::kTileM);
+  // all M-tiles per column sweep when A (M x K bytes) fits in half of L2
+  p.group_m = a.M * a.K <= (64ll << 20) ? p.m_tiles : 8;
   const int tiles = p.m_tiles * p.n_tiles;
   const int per_unit = PAIR ? 2 : 1;
   const int max_units = sm_count() / per_unit;

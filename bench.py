@@ -40,9 +40,10 @@ FALLBACK_BF16_TFLOPS = 1590.0
 INT8_PER_BF16 = 2.0  # nominal dense int8 : bf16 tensor throughput (4.5 : 2.25 POPS)
 
 # DRAM bytes per launch from ncu (dram__bytes_read.sum + dram__bytes_write.sum),
-# keyed by kernel and shape, valid only for the kernel source they were taken on.
-NCU_TRAFFIC = {}
-NCU_TRAFFIC_SOURCE_SHA = {}
+# averaged over the three GEMM launches of one Z-Image step, valid only for the
+# kernel source they were taken on (first 16 hex digits of its sha256).
+NCU_TRAFFIC = {"int8_gemm_tcgen05": (120.5e6 + 102.5e6 + 152.4e6) / 3}
+NCU_TRAFFIC_SOURCE_SHA = {"int8_gemm_tcgen05": "7e9889ec198664ca"}
 
 
 def source_sha(rel: str) -> str:
@@ -140,6 +141,7 @@ def init_pg(world: int, backend: str):
 
 
 def max_over_ranks(value: float, world: int, device) -> float:
+    """The largest `value` over all ranks (host-side timing plumbing)."""
     if world == 1:
         return value
     import torch
@@ -147,6 +149,15 @@ def max_over_ranks(value: float, world: int, device) -> float:
     t = torch.tensor([value], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def weak_scaling_throughput(ops_per_rank_step: float, steps: int, local_ms: float, world: int,
+                            device) -> tuple[float, float]:
+    """Whole-job throughput of weak-scaled replicas: every rank processed
+    `steps` steps of `ops_per_rank_step` operations; the job took as long as the
+    slowest rank.  Returns (TOP/s, max-over-ranks milliseconds)."""
+    total_ms = max_over_ranks(local_ms, world, device)
+    return ops_per_rank_step * steps * world / (total_ms * 1e-3) / 1e12, total_ms
 
 
 def barrier(world: int):
@@ -310,10 +321,8 @@ def run_ours(args, lins):
     rqa_ms = np.array([[r[i][0].elapsed_time(r[i][1]) for i in range(n_lin)] for r in recs])
     gemm_ms = np.array([[r[i][1].elapsed_time(r[i][2]) for i in range(n_lin)] for r in recs])
     step_ms = np.array([r[0][0].elapsed_time(r[-1][2]) for r in recs])
-    local_total_ms = float(step_ms.sum())
-    total_ms = max_over_ranks(local_total_ms, world, dev)
     ops_step = sum(2.0 * L["lin"].M * L["lin"].N * L["lin"].K for L in layers)
-    value = ops_step * args.steps * world / (total_ms * 1e-3) / 1e12
+    value, total_ms = weak_scaling_throughput(ops_step, args.steps, float(step_ms.sum()), world, dev)
 
     gemm_mean = gemm_ms.mean(axis=0)
     gemm_ops = np.array([2.0 * L["lin"].M * L["lin"].N * L["lin"].K for L in layers])
@@ -360,8 +369,7 @@ def run_ours(args, lins):
         torch.cuda.synchronize()
         if k:  # first pass warms the pinned-copy path
             e2e_ms.append(e0.elapsed_time(e1))
-    e2e_total = max_over_ranks(float(np.mean(e2e_ms)), world, dev)
-    e2e_value = ops_step * world / (e2e_total * 1e-3) / 1e12
+    e2e_value, e2e_total = weak_scaling_throughput(ops_step, 1, float(np.mean(e2e_ms)), world, dev)
 
     if rank != 0:
         return 0
