@@ -429,9 +429,10 @@ cudaError_t launch_int8_gemm(const GemmArgs& a, cudaStream_t stream) {
   p.n_tiles = static_cast<int>((a.N + BN - 1) / BN);
   p.per_channel_scale = a.s_w_len > 1 ? 1 : 0;
   p.out_s32 = a.out_s32 ? 1 : 0;
-  // CTA pairs (256-row tiles) once there is more than one 128-row block of tokens
-  if (a.M > BM) return launch_variant<true>(a, p, stream);
-  return launch_variant<false>(a, p, stream);
+  // few tokens: the weight-streaming swap-AB kernel; otherwise CTA pairs
+  // (256-row tiles) once there is more than one 128-row block of tokens
+  if (a.M <= BM) return launch_int8_gemm_skinny(a, stream);
+  return launch_variant<true>(a, p, stream);
 }
 
 }  // namespace convrot

@@ -51,6 +51,9 @@ struct GemmArgs {
 // cudaErrorInvalidValue if a tensor map cannot be encoded.
 cudaError_t launch_int8_gemm(const GemmArgs& a, cudaStream_t stream);
 
+// The few-token variant (M <= 128): swap-AB with the K split over a cluster.
+cudaError_t launch_int8_gemm_skinny(const GemmArgs& a, cudaStream_t stream);
+
 // Reads and clears the current device's kernel status word (0 = fine).
 cudaError_t read_and_clear_status(unsigned int* status, cudaStream_t stream);
 

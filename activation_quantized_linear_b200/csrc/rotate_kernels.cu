@@ -123,10 +123,12 @@ __device__ __forceinline__ void load_i8_32(const int8_t* p, uint64_t (&P)[kPairs
 //   G == 256: bits 5..7 after one exchange through shared memory: the 8 lanes
 //   of a group each write their 32 elements as 8 slots of 16 bytes and read
 //   slot t (elements 4t .. 4t + 3) of every lane of the group; slot m of lane
-//   s sits at 8 s + (m ^ s), so the 8 lanes of a quarter-warp (one group) hit
-//   8 distinct bank quads on both sides.  Afterwards lane t holds in
+//   s sits at 9 s + m (rows padded to 9 slots), so the 8 lanes of a
+//   quarter-warp (one group) hit 8 distinct bank quads on both sides, and every
+//   address is a per-lane base plus a constant.  Afterwards lane t holds in
 //   P[2 s + q] the elements (32 s + 4t + 2q, 32 s + 4t + 2q + 1), s = 0..7.
-constexpr int kXchBytesPerWarp = 4 * 64 * 16;  // 4 groups x 64 slots
+constexpr int kXchGroupBytes = 8 * 9 * 16;
+constexpr int kXchBytesPerWarp = 4 * kXchGroupBytes;  // 4 groups
 
 template <int G>
 __device__ __forceinline__ void fwht32(uint64_t (&P)[kPairs], uint32_t xch, uint32_t lane) {
@@ -159,12 +161,13 @@ __device__ __forceinline__ void fwht32(uint64_t (&P)[kPairs], uint32_t xch, uint
   }
   if constexpr (G == 256) {
     const uint32_t t = lane & 7;
-    const uint32_t g = xch + (lane >> 3) * (64 * 16);
+    const uint32_t g = xch + (lane >> 3) * kXchGroupBytes;
+    const uint32_t wbase = g + 144 * t, rbase = g + 16 * t;
 #pragma unroll
-    for (int m = 0; m < 8; ++m) sts128(g + 16 * (8 * t + (m ^ t)), P[2 * m], P[2 * m + 1]);
+    for (int m = 0; m < 8; ++m) sts128(wbase + 16 * m, P[2 * m], P[2 * m + 1]);
     __syncwarp();
 #pragma unroll
-    for (int s = 0; s < 8; ++s) lds128(g + 16 * (8 * s + (t ^ s)), P[2 * s], P[2 * s + 1]);
+    for (int s = 0; s < 8; ++s) lds128(rbase + 144 * s, P[2 * s], P[2 * s + 1]);
     __syncwarp();
 #pragma unroll
     for (int h = 1; h < 8; h <<= 1) {  // bits 5..7: across source lanes
@@ -245,8 +248,12 @@ __device__ __forceinline__ uint32_t bf16x2_exact_product(uint64_t s2, uint64_t v
   const uint64_t p = mulrz2(s2, v);
   const uint64_t e = fma2(s2, v, p ^ 0x8000000080000000ull);  // exact remainder s*v - p
   uint32_t lo = static_cast<uint32_t>(p), hi = static_cast<uint32_t>(p >> 32);
-  lo |= (static_cast<uint32_t>(e) << 1) != 0u ? 1u : 0u;
-  hi |= (static_cast<uint32_t>(e >> 32) << 1) != 0u ? 1u : 0u;
+  // the remainder is +0 exactly when the product is exact (x - x rounds to +0)
+  asm("{\n\t.reg .pred q;\n\t"
+      "setp.ne.b32 q, %2, 0;\n\t@q or.b32 %0, %0, 1;\n\t"
+      "setp.ne.b32 q, %3, 0;\n\t@q or.b32 %1, %1, 1;\n\t}"
+      : "+r"(lo), "+r"(hi)
+      : "r"(static_cast<uint32_t>(e)), "r"(static_cast<uint32_t>(e >> 32)));
   const __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(lo), __uint_as_float(hi));
   return *reinterpret_cast<const uint32_t*>(&h);
 }
@@ -311,15 +318,14 @@ __global__ void __launch_bounds__(1024) rotate_quant_act_hadamard(
   const bool ok = row_ok && t < nch;  // whole groups agree (K % G == 0)
   const uint32_t xch = smem_addr(xch_all) + warp * xch_bytes_per_warp<G>();
 
+  // Lanes without a chunk (the row's tail, or rows past M) load a valid chunk
+  // instead of zeros; whole groups share `ok`, and their maxima are dropped.
   uint64_t P[kPairs];
-  if (ok) {
-    load_bf16_32(x + row * K + static_cast<int64_t>(t) * kVec, P);
-  } else {
-#pragma unroll
-    for (int i = 0; i < kPairs; ++i) P[i] = 0;
-  }
+  const int64_t src_row = row_ok ? row : 0;
+  const int src_t = t < nch ? t : 0;
+  load_bf16_32(x + src_row * K + static_cast<int64_t>(src_t) * kVec, P);
   fwht32<G>(P, xch, lane);
-  float amax = warp_max(absmax32(P));
+  float amax = warp_max(ok ? absmax32(P) : 0.f);
   if (team_warps > 1) {
     if (lane == 0) red[warp] = amax;
     __syncthreads();
@@ -347,7 +353,7 @@ __global__ void __launch_bounds__(1024) rotate_quant_act_hadamard(
 enum FlatMode { kFlatAbsmax = 0, kFlatQuant = 1, kFlatDequant = 2 };
 
 template <int G, int MODE, bool PER_ROW_SCALE>
-__global__ void __launch_bounds__(256) hadamard_flat(const void* __restrict__ in, int64_t nchunks,
+__global__ void __launch_bounds__(256, 4) hadamard_flat(const void* __restrict__ in, int64_t nchunks,
                                                      int64_t chunks_per_row,
                                                      const float* __restrict__ scale,
                                                      void* __restrict__ out,
@@ -359,22 +365,19 @@ __global__ void __launch_bounds__(256) hadamard_flat(const void* __restrict__ in
   const uint32_t xch = smem_addr(xch_all) + (threadIdx.x >> 5) * xch_bytes_per_warp<G>();
   constexpr float norm = Norm<G>::value;
 
+  // lanes past the end load chunk 0 (whole groups share `ok`) and are dropped
   uint64_t P[kPairs];
-  if (ok) {
-    if constexpr (MODE == kFlatDequant) {
-      load_i8_32(static_cast<const int8_t*>(in) + c * kVec, P);
-    } else {
-      load_bf16_32(static_cast<const uint16_t*>(in) + c * kVec, P);
-    }
+  const int64_t src = ok ? c : 0;
+  if constexpr (MODE == kFlatDequant) {
+    load_i8_32(static_cast<const int8_t*>(in) + src * kVec, P);
   } else {
-#pragma unroll
-    for (int i = 0; i < kPairs; ++i) P[i] = 0;
+    load_bf16_32(static_cast<const uint16_t*>(in) + src * kVec, P);
   }
   fwht32<G>(P, xch, lane);
 
   if constexpr (MODE == kFlatAbsmax) {
     __shared__ float red[8];
-    const float amax = warp_max(absmax32(P));
+    const float amax = warp_max(ok ? absmax32(P) : 0.f);
     if (lane == 0) red[threadIdx.x >> 5] = amax;
     __syncthreads();
     if (threadIdx.x == 0) {

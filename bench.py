@@ -409,6 +409,67 @@ def run_ours(args, lins):
     return 0
 
 
+def run_sweep(args):
+    """Per-shape kernel times of the group-size / skinny-M sweep (K = N = 4096,
+    G in {4, 16, 64, 256}, M in {1, 16, 128, 1024, 8192}) and of the standalone
+    decode of a [12288, 3072] int8 weight at each G; one JSON line."""
+    import torch
+
+    import activation_quantized_linear_b200 as cr
+    torch.cuda.set_device(0)
+    hbm_gbs, bf16_tflops, _, _ = load_peaks()
+    int8_peak = bf16_tflops * INT8_PER_BF16
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    flush_rd = torch.ones(64 << 20, dtype=torch.float32, device="cuda")
+
+    def timed(fn, n):
+        ts = []
+        for k in range(n + 3):
+            flush.fill_(k & 0xFF)
+            flush_rd.sum()
+            torch.cuda._sleep(400_000)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            if k >= 3:
+                ts.append(e0.elapsed_time(e1))
+        return statistics.median(ts)
+
+    rows = []
+    for G in workloads.GROUP_SIZES:
+        rot = cr.Rotation(workloads.sylvester_rotation(G))
+        for M in (1, 16, 128, 1024, 8192):
+            lin = workloads.Linear("sweep", M, 4096, 4096, G=G)
+            inp = workloads.make_layer_inputs(lin, 4)
+            Wq, s_w = cr.quantize_weight(inp.W.cuda(), rot)
+            x, bias = inp.x.cuda(), inp.bias.cuda()
+            xq, s_tok = cr.rotate_quant_act(x, rot)
+            y = cr.int8_gemm(xq, s_tok, Wq, s_w, bias)
+            t_r = timed(lambda: cr.rotate_quant_act(x, rot, xq=xq, s_tok=s_tok), args.steps)
+            t_g = timed(lambda: cr.int8_gemm(xq, s_tok, Wq, s_w, bias, out=y), args.steps)
+            ops = 2.0 * M * 4096 * 4096
+            gemm_bytes = M * 4096 + 4096 * 4096 + 2 * M * 4096
+            rows.append({"G": G, "M": M, "rotate_ms": t_r, "rotate_GBps": (3 * M * 4096 + 4 * M) / t_r / 1e6,
+                         "gemm_ms": t_g, "gemm_TOPS": ops / t_g / 1e9,
+                         "gemm_frac_int8_peak": ops / t_g / 1e9 / int8_peak,
+                         "gemm_GBps": gemm_bytes / t_g / 1e6,
+                         "gemm_frac_hbm": gemm_bytes / t_g / 1e6 / hbm_gbs})
+    dec = []
+    N, K = workloads.DEROTATE_SWEEP_SHAPE
+    for G in workloads.GROUP_SIZES:
+        rot = cr.Rotation(workloads.sylvester_rotation(G))
+        Wq = torch.randint(-127, 128, (N, K), dtype=torch.int8, device="cuda")
+        s_w = torch.tensor([1e-3], device="cuda")
+        out = torch.empty((N, K), dtype=torch.bfloat16, device="cuda")
+        t = timed(lambda: cr.dequant_derotate(Wq, s_w, rot, out=out), args.steps)
+        dec.append({"G": G, "ms": t, "GBps": 3 * N * K / t / 1e6, "frac_hbm": 3 * N * K / t / 1e6 / hbm_gbs})
+    print(json.dumps({"sweep": "group_size_and_skinny_M", "linears": rows, "decode_12288x3072": dec,
+                      "peaks": {"hbm_gbs": hbm_gbs, "int8_tops": int8_peak}}))
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -420,9 +481,13 @@ def main():
     ap.add_argument("--ref-rows", type=int, default=64)
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep", action="store_true",
+                    help="time the group-size / skinny-M sweep and the decode sweep instead")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
+    if args.sweep:
+        return run_sweep(args)
     lins = workloads.WORKLOADS[args.workload]
     if args.impl == "reference":
         return run_reference(args, lins)
