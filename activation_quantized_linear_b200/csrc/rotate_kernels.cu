@@ -42,11 +42,30 @@ struct Norm {  // 1 / sqrt(G), exact
 // ---------------------------------------------------------------- packed pairs
 // sm_100 executes two float32 operations per instruction on a 64-bit register
 // pair; the butterflies, the scaling and the code rounding use these forms.
+// A pair is a 64-bit register pair; pack and unpack only name its halves.
 __device__ __forceinline__ uint64_t pk(float lo, float hi) {
-  return (static_cast<uint64_t>(__float_as_uint(hi)) << 32) | __float_as_uint(lo);
+  uint64_t d;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(lo), "f"(hi));
+  return d;
 }
-__device__ __forceinline__ float plo(uint64_t p) { return __uint_as_float(static_cast<uint32_t>(p)); }
-__device__ __forceinline__ float phi(uint64_t p) { return __uint_as_float(static_cast<uint32_t>(p >> 32)); }
+__device__ __forceinline__ uint64_t pku(uint32_t lo, uint32_t hi) {
+  uint64_t d;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "r"(lo), "r"(hi));
+  return d;
+}
+__device__ __forceinline__ void unpk(uint64_t p, uint32_t& lo, uint32_t& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(lo), "=r"(hi) : "l"(p));
+}
+__device__ __forceinline__ float plo(uint64_t p) {
+  uint32_t lo, hi;
+  unpk(p, lo, hi);
+  return __uint_as_float(lo);
+}
+__device__ __forceinline__ float phi(uint64_t p) {
+  uint32_t lo, hi;
+  unpk(p, lo, hi);
+  return __uint_as_float(hi);
+}
 __device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
   uint64_t d;
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
@@ -80,31 +99,24 @@ __device__ __forceinline__ void lds128(uint32_t addr, uint64_t& a, uint64_t& b) 
 }
 
 // ---------------------------------------------------------------- loads
-// 32 bf16 at p (16-byte aligned) -> P[i] = (p[2i], p[2i + 1]).
-__device__ __forceinline__ void load_bf16_32(const uint16_t* p, uint64_t (&P)[kPairs]) {
-  const uint4* q = reinterpret_cast<const uint4*>(p);
-  uint4 u[4];
-#pragma unroll
-  for (int j = 0; j < 4; ++j) u[j] = __ldg(q + j);
+// raw words -> P[i] = (p[2i], p[2i + 1]) as floats.
+__device__ __forceinline__ void widen_bf16_32(const uint4 (&u)[4], uint64_t (&P)[kPairs]) {
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
     const uint32_t w[4] = {u[j].x, u[j].y, u[j].z, u[j].w};
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-      P[4 * j + k] = pk(__uint_as_float(w[k] << 16), __uint_as_float(w[k] & 0xffff0000u));
+      P[4 * j + k] = pku(w[k] << 16, w[k] & 0xffff0000u);
     }
   }
 }
 
-// 32 int8 at p (16-byte aligned) -> P[i] = (p[2i], p[2i + 1]).
-__device__ __forceinline__ void load_i8_32(const int8_t* p, uint64_t (&P)[kPairs]) {
-  const int4* q = reinterpret_cast<const int4*>(p);
-  int4 u[2];
-#pragma unroll
-  for (int j = 0; j < 2; ++j) u[j] = __ldg(q + j);
+// raw int8 words -> P[i] = (p[2i], p[2i + 1]) as floats.
+__device__ __forceinline__ void widen_i8_32(const uint4 (&u)[2], uint64_t (&P)[kPairs]) {
 #pragma unroll
   for (int j = 0; j < 2; ++j) {
-    const int w[4] = {u[j].x, u[j].y, u[j].z, u[j].w};
+    const int w[4] = {static_cast<int>(u[j].x), static_cast<int>(u[j].y),
+                      static_cast<int>(u[j].z), static_cast<int>(u[j].w)};
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       P[8 * j + 2 * k] = pk(static_cast<float>(static_cast<int8_t>(w[k])),
@@ -199,8 +211,10 @@ __device__ __forceinline__ void store_code_bytes(int8_t* base, const uint64_t (&
   uint32_t w[8];
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
-    w[j] = pack4(static_cast<uint32_t>(R[2 * j]), static_cast<uint32_t>(R[2 * j] >> 32),
-                 static_cast<uint32_t>(R[2 * j + 1]), static_cast<uint32_t>(R[2 * j + 1] >> 32));
+    uint32_t a0, a1, b0, b1;
+    unpk(R[2 * j], a0, a1);
+    unpk(R[2 * j + 1], b0, b1);
+    w[j] = pack4(a0, a1, b0, b1);
   }
   if constexpr (G == 256) {
     const uint32_t t = lane & 7;
@@ -246,14 +260,17 @@ __device__ __forceinline__ void store_codes32_div(int8_t* base, const uint64_t (
 // rounding that to bf16 is the correctly rounded result.
 __device__ __forceinline__ uint32_t bf16x2_exact_product(uint64_t s2, uint64_t v) {
   const uint64_t p = mulrz2(s2, v);
-  const uint64_t e = fma2(s2, v, p ^ 0x8000000080000000ull);  // exact remainder s*v - p
-  uint32_t lo = static_cast<uint32_t>(p), hi = static_cast<uint32_t>(p >> 32);
+  uint32_t lo, hi;
+  unpk(p, lo, hi);
+  const uint64_t e = fma2(s2, v, pku(lo ^ 0x80000000u, hi ^ 0x80000000u));  // exact s*v - p
+  uint32_t e_lo, e_hi;
+  unpk(e, e_lo, e_hi);
   // the remainder is +0 exactly when the product is exact (x - x rounds to +0)
   asm("{\n\t.reg .pred q;\n\t"
       "setp.ne.b32 q, %2, 0;\n\t@q or.b32 %0, %0, 1;\n\t"
       "setp.ne.b32 q, %3, 0;\n\t@q or.b32 %1, %1, 1;\n\t}"
       : "+r"(lo), "+r"(hi)
-      : "r"(static_cast<uint32_t>(e)), "r"(static_cast<uint32_t>(e >> 32)));
+      : "r"(e_lo), "r"(e_hi));
   const __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(lo), __uint_as_float(hi));
   return *reinterpret_cast<const uint32_t*>(&h);
 }
@@ -302,47 +319,114 @@ __host__ __device__ constexpr int xch_bytes_per_warp() {
 // 32-element chunk per lane, all loads issued before any arithmetic.  The
 // token's rotated row stays in registers between the absmax and the pack.
 // ===========================================================================
+// Per-lane 16-byte asynchronous copies global -> shared (bypassing L1).
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+// A warp stages 32 consecutive chunks of kParts 16-byte units each (bf16:
+// 4, int8: 2) in a slot of its own.  Copy j of lane i moves unit j * 32 + i, so
+// each copy instruction reads 512 contiguous bytes; unit u sits at position
+// stage_pos(u), which rotates every row of 8 units by (u >> 3) so that the
+// copies' stores and the lanes' reads of their own units (kParts * lane + k)
+// both fall in distinct banks.
+__device__ __forceinline__ uint32_t stage_pos(uint32_t u) {
+  return (u & ~7u) | ((u + (u >> 3)) & 7u);
+}
+
+// chunks chunk0 .. chunk0 + 31 of a row whose chunk c starts at
+// base + c * kParts * 16; chunks at or past `nvalid` copy chunk 0 instead
+template <int kParts>
+__device__ __forceinline__ void stage_chunks(uint32_t slot, uint32_t lane, const uint8_t* base,
+                                             int64_t chunk0, int64_t nvalid) {
+#pragma unroll
+  for (int j = 0; j < kParts; ++j) {
+    const uint32_t u = j * 32 + lane;
+    const int64_t c = chunk0 + u / kParts;
+    cp_async16(slot + stage_pos(u) * 16,
+               base + ((c < nvalid ? c : 0) * kParts + u % kParts) * 16);
+  }
+  cp_async_commit();
+}
+
+template <int kParts>
+__device__ __forceinline__ void unstage_chunk(uint32_t slot, uint32_t lane, uint4 (&v)[kParts]) {
+#pragma unroll
+  for (int k = 0; k < kParts; ++k) {
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v[k].x), "=r"(v[k].y), "=r"(v[k].z), "=r"(v[k].w)
+                 : "r"(slot + stage_pos(kParts * lane + k) * 16)
+                 : "memory");
+  }
+}
+
+constexpr int kStageBytesPerWarp = 32 * kVec * 2;
+
 template <int G>
 __global__ void __launch_bounds__(1024) rotate_quant_act_hadamard(
     const uint16_t* __restrict__ x, int64_t M, int K, int team_warps, int rows_per_cta,
     int8_t* __restrict__ xq, float* __restrict__ s_tok) {
-  extern __shared__ __align__(16) uint8_t xch_all[];
-  __shared__ float red[32];
+  extern __shared__ __align__(16) uint8_t smem_all[];
+  __shared__ float red[2][32];
   const int warp = threadIdx.x >> 5;
   const uint32_t lane = threadIdx.x & 31;
   const int team = warp / team_warps;
-  const int t = (warp % team_warps) * 32 + static_cast<int>(lane);  // chunk within the token
-  const int64_t row = static_cast<int64_t>(blockIdx.x) * rows_per_cta + team;
-  const bool row_ok = row < M;  // uniform over the team
+  const int t0 = (warp % team_warps) * 32;
+  const int t = t0 + static_cast<int>(lane);  // chunk within the token
   const int nch = K / kVec;
-  const bool ok = row_ok && t < nch;  // whole groups agree (K % G == 0)
-  const uint32_t xch = smem_addr(xch_all) + warp * xch_bytes_per_warp<G>();
-
-  // Lanes without a chunk (the row's tail, or rows past M) load a valid chunk
-  // instead of zeros; whole groups share `ok`, and their maxima are dropped.
-  uint64_t P[kPairs];
-  const int64_t src_row = row_ok ? row : 0;
-  const int src_t = t < nch ? t : 0;
-  load_bf16_32(x + src_row * K + static_cast<int64_t>(src_t) * kVec, P);
-  fwht32<G>(P, xch, lane);
-  float amax = warp_max(ok ? absmax32(P) : 0.f);
-  if (team_warps > 1) {
-    if (lane == 0) red[warp] = amax;
-    __syncthreads();
-    amax = 0.f;
-    for (int k = 0; k < team_warps; ++k) amax = fmaxf(amax, red[team * team_warps + k]);
-  }
-  if (!ok) return;
-
+  const int nwarps = blockDim.x >> 5;
+  const uint32_t slot = smem_addr(smem_all) + warp * kStageBytesPerWarp;
+  const uint32_t xch = smem_addr(smem_all) + nwarps * kStageBytesPerWarp + warp * xch_bytes_per_warp<G>();
+  const int64_t blocks = (M + rows_per_cta - 1) / rows_per_cta;
   constexpr float norm = Norm<G>::value;
-  const float s = (amax * norm) / 127.f;  // s_tok = max |x_rot| / 127
-  if (t == 0) s_tok[row] = s;
-  const float mul = norm * (s > 0.f ? 1.f / s : 0.f);  // exact scaling: norm is a power of two
-  int8_t* dst = xq + row * K + static_cast<int64_t>(t) * kVec;
-  if (mul <= 3.0e38f) {
-    store_codes32<G>(dst, P, mul, lane);
-  } else {
-    store_codes32_div<G>(dst, P, norm, s, lane);
+
+  // The CTA walks row blocks blockIdx.x, blockIdx.x + gridDim.x, ...; the next
+  // block's chunks are copied into shared memory while this one is transformed.
+  // Lanes without a chunk (the row's tail, rows past M) are given chunk 0 of a
+  // valid row instead; whole groups share `ok`, and their maxima are dropped.
+  const int bar_id = 1 + team, bar_threads = team_warps * 32;
+  int64_t rb = blockIdx.x;
+  if (rb < blocks) {
+    const int64_t r = rb * rows_per_cta + team;
+    stage_chunks<4>(slot, lane, reinterpret_cast<const uint8_t*>(x + (r < M ? r : 0) * K), t0, nch);
+  }
+  for (int it = 0; rb < blocks; rb += gridDim.x, ++it) {
+    const int64_t row = rb * rows_per_cta + team;
+    const bool row_ok = row < M;  // uniform over the team
+    const bool ok = row_ok && t < nch;
+    uint4 u[4];
+    cp_async_wait_all();
+    __syncwarp();  // the lanes' copies landed: every lane's units are visible
+    unstage_chunk<4>(slot, lane, u);
+    uint64_t P[kPairs];
+    widen_bf16_32(u, P);
+    __syncwarp();  // every lane has read its units before the slot is refilled
+    if (rb + gridDim.x < blocks) {
+      const int64_t r = (rb + gridDim.x) * rows_per_cta + team;
+      stage_chunks<4>(slot, lane, reinterpret_cast<const uint8_t*>(x + (r < M ? r : 0) * K), t0, nch);
+    }
+    fwht32<G>(P, xch, lane);
+    float amax = warp_max(ok ? absmax32(P) : 0.f);
+    if (team_warps > 1) {
+      float* rb_red = red[it & 1];
+      if (lane == 0) rb_red[warp] = amax;
+      // the team's warps only: teams of one CTA run independently
+      asm volatile("bar.sync %0, %1;" ::"r"(bar_id), "r"(bar_threads) : "memory");
+      amax = 0.f;
+      for (int k = 0; k < team_warps; ++k) amax = fmaxf(amax, rb_red[team * team_warps + k]);
+    }
+    if (!ok) continue;
+    const float sc = (amax * norm) / 127.f;  // s_tok = max |x_rot| / 127
+    if (t == 0) s_tok[row] = sc;
+    const float mul = norm * (sc > 0.f ? 1.f / sc : 0.f);  // exact scaling: norm is a power of two
+    int8_t* dst = xq + row * K + static_cast<int64_t>(t) * kVec;
+    if (mul <= 3.0e38f) {
+      store_codes32<G>(dst, P, mul, lane);
+    } else {
+      store_codes32_div<G>(dst, P, norm, sc, lane);
+    }
   }
 }
 
@@ -353,53 +437,81 @@ __global__ void __launch_bounds__(1024) rotate_quant_act_hadamard(
 enum FlatMode { kFlatAbsmax = 0, kFlatQuant = 1, kFlatDequant = 2 };
 
 template <int G, int MODE, bool PER_ROW_SCALE>
-__global__ void __launch_bounds__(256, 4) hadamard_flat(const void* __restrict__ in, int64_t nchunks,
+__global__ void __launch_bounds__(256, MODE == kFlatDequant ? 3 : 4) hadamard_flat(const void* __restrict__ in, int64_t nchunks,
                                                      int64_t chunks_per_row,
                                                      const float* __restrict__ scale,
                                                      void* __restrict__ out,
                                                      unsigned int* __restrict__ absmax_bits) {
-  extern __shared__ __align__(16) uint8_t xch_all[];
+  constexpr int kParts = MODE == kFlatDequant ? 2 : 4;  // 16-byte parts of a chunk
+  extern __shared__ __align__(16) uint8_t smem_all[];
   const uint32_t lane = threadIdx.x & 31;
-  const int64_t c = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const bool ok = c < nchunks;  // whole groups agree: nchunks % (G / 32) == 0
-  const uint32_t xch = smem_addr(xch_all) + (threadIdx.x >> 5) * xch_bytes_per_warp<G>();
+  const int warp = threadIdx.x >> 5;
+  const uint32_t slot = smem_addr(smem_all) + warp * (kParts * 512);
+  const uint32_t xch =
+      smem_addr(smem_all) + (blockDim.x >> 5) * (kParts * 512) + warp * xch_bytes_per_warp<G>();
+  const int64_t blocks = (nchunks + blockDim.x - 1) / blockDim.x;
+  const uint8_t* src = static_cast<const uint8_t*>(in);
   constexpr float norm = Norm<G>::value;
 
-  // lanes past the end load chunk 0 (whole groups share `ok`) and are dropped
-  uint64_t P[kPairs];
-  const int64_t src = ok ? c : 0;
-  if constexpr (MODE == kFlatDequant) {
-    load_i8_32(static_cast<const int8_t*>(in) + src * kVec, P);
-  } else {
-    load_bf16_32(static_cast<const uint16_t*>(in) + src * kVec, P);
+  // Chunk c = b * blockDim.x + thread for blocks b = blockIdx.x, + gridDim.x, ...;
+  // the next block's chunk is copied into shared memory while this one is
+  // transformed.  Lanes past the end copy chunk 0 (whole groups share `ok`)
+  // and are dropped.
+  auto stage = [&](int64_t b) {
+    stage_chunks<kParts>(slot, lane, src, b * blockDim.x + warp * 32, nchunks);
+  };
+  float mul = 0.f, s = 0.f, run_max = 0.f;
+  if constexpr (MODE == kFlatQuant) {
+    s = __uint_as_float(*absmax_bits) / 127.f;
+    mul = s > 0.f ? norm * (1.f / s) : 0.f;
   }
-  fwht32<G>(P, xch, lane);
+  int64_t b = blockIdx.x;
+  if (b < blocks) stage(b);
+  for (; b < blocks; b += gridDim.x) {
+    const int64_t c = b * blockDim.x + threadIdx.x;
+    const bool ok = c < nchunks;
+    uint4 u[kParts];
+    cp_async_wait_all();
+    __syncwarp();  // the lanes' copies landed: every lane's units are visible
+    unstage_chunk<kParts>(slot, lane, u);
+    uint64_t P[kPairs];
+    if constexpr (MODE == kFlatDequant) {
+      widen_i8_32(u, P);
+    } else {
+      widen_bf16_32(u, P);
+    }
+    __syncwarp();  // every lane has read its units before the slot is refilled
+    if (b + gridDim.x < blocks) stage(b + gridDim.x);
+    fwht32<G>(P, xch, lane);
 
+    if constexpr (MODE == kFlatAbsmax) {
+      if (ok) run_max = fmaxf(run_max, absmax32(P));
+    } else if constexpr (MODE == kFlatQuant) {
+      if (ok) {
+        int8_t* dst = static_cast<int8_t*>(out) + c * kVec;
+        if (mul <= 3.0e38f) {
+          store_codes32<G>(dst, P, mul, lane);
+        } else {
+          store_codes32_div<G>(dst, P, norm, s, lane);
+        }
+      }
+    } else {
+      if (ok) {
+        const float sw = PER_ROW_SCALE ? scale[c / chunks_per_row] : scale[0];
+        store_bf16_32<G>(static_cast<uint16_t*>(out) + c * kVec, P, sw * norm, lane);
+      }
+    }
+  }
   if constexpr (MODE == kFlatAbsmax) {
     __shared__ float red[8];
-    const float amax = warp_max(ok ? absmax32(P) : 0.f);
-    if (lane == 0) red[threadIdx.x >> 5] = amax;
+    const float amax = warp_max(run_max);
+    if (lane == 0) red[warp] = amax;
     __syncthreads();
     if (threadIdx.x == 0) {
       float m = 0.f;
       for (int k = 0; k < static_cast<int>(blockDim.x >> 5); ++k) m = fmaxf(m, red[k]);
       atomicMax(absmax_bits, __float_as_uint(m * norm));  // non-negative: bit order = value order
     }
-  } else if constexpr (MODE == kFlatQuant) {
-    if (!ok) return;
-    const float a = __uint_as_float(*absmax_bits);
-    const float s = a / 127.f;
-    const float mul = s > 0.f ? norm * (1.f / s) : 0.f;
-    int8_t* dst = static_cast<int8_t*>(out) + c * kVec;
-    if (mul <= 3.0e38f) {
-      store_codes32<G>(dst, P, mul, lane);
-    } else {
-      store_codes32_div<G>(dst, P, norm, s, lane);
-    }
-  } else {
-    if (!ok) return;
-    const float sw = PER_ROW_SCALE ? scale[c / chunks_per_row] : scale[0];
-    store_bf16_32<G>(static_cast<uint16_t*>(out) + c * kVec, P, sw * norm, lane);
   }
 }
 
@@ -541,10 +653,18 @@ cudaError_t rqa_hadamard(const uint16_t* x, int64_t M, int64_t K, int8_t* xq, fl
   const int team_warps = (nch + 31) / 32;
   const int rows_per_cta = team_warps >= 8 ? 1 : 8 / team_warps;
   const int warps = team_warps * rows_per_cta;
-  const size_t smem = static_cast<size_t>(warps) * xch_bytes_per_warp<G>();
+  const size_t smem = static_cast<size_t>(warps) * (kStageBytesPerWarp + xch_bytes_per_warp<G>());
   cudaError_t e = allow_smem(rotate_quant_act_hadamard<G>, smem);
   if (e != cudaSuccess) return e;
-  const int64_t grid = (M + rows_per_cta - 1) / rows_per_cta;
+  // enough CTAs to fill every SM (register-limited occupancy), each looping
+  // over row blocks with a one-block-ahead prefetch
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, rotate_quant_act_hadamard<G>,
+                                                    32 * warps, smem);
+  if (e != cudaSuccess) return e;
+  const int64_t blocks = (M + rows_per_cta - 1) / rows_per_cta;
+  const int64_t cap = static_cast<int64_t>(sm_count()) * (per_sm > 0 ? per_sm : 1);
+  const int64_t grid = blocks < cap ? blocks : cap;
   rotate_quant_act_hadamard<G><<<static_cast<unsigned>(grid), 32 * warps, smem, stream>>>(
       x, M, static_cast<int>(K), team_warps, rows_per_cta, xq, s_tok);
   return cudaGetLastError();
@@ -555,10 +675,18 @@ cudaError_t flat_launch(const void* in, int64_t nchunks, int64_t chunks_per_row,
                         const float* scale, void* out, unsigned int* absmax_bits,
                         cudaStream_t stream) {
   constexpr int kThreadsFlat = 256;
-  const size_t smem = (kThreadsFlat / 32) * xch_bytes_per_warp<G>();
+  constexpr int kParts = MODE == kFlatDequant ? 2 : 4;
+  const size_t smem = (kThreadsFlat / 32) * (kParts * 512 + xch_bytes_per_warp<G>());
   cudaError_t e = allow_smem(hadamard_flat<G, MODE, PER_ROW>, smem);
   if (e != cudaSuccess) return e;
-  int64_t grid = (nchunks + kThreadsFlat - 1) / kThreadsFlat;  // one chunk per thread
+  // one chunk per thread and block; enough CTAs to fill every SM, each looping
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, hadamard_flat<G, MODE, PER_ROW>,
+                                                    kThreadsFlat, smem);
+  if (e != cudaSuccess) return e;
+  const int64_t cap = static_cast<int64_t>(sm_count()) * (per_sm > 0 ? per_sm : 1);
+  int64_t grid = (nchunks + kThreadsFlat - 1) / kThreadsFlat;
+  if (grid > cap) grid = cap;
   if (grid < 1) grid = 1;
   hadamard_flat<G, MODE, PER_ROW><<<static_cast<unsigned>(grid), kThreadsFlat, smem, stream>>>(
       in, nchunks, chunks_per_row, scale, out, absmax_bits);
