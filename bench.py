@@ -42,8 +42,8 @@ INT8_PER_BF16 = 2.0  # nominal dense int8 : bf16 tensor throughput (4.5 : 2.25 P
 # DRAM bytes per launch from ncu (dram__bytes_read.sum + dram__bytes_write.sum),
 # averaged over the three GEMM launches of one Z-Image step, valid only for the
 # kernel source they were taken on (first 16 hex digits of its sha256).
-NCU_TRAFFIC = {"int8_gemm_tcgen05": (120.5e6 + 102.5e6 + 152.4e6) / 3}
-NCU_TRAFFIC_SOURCE_SHA = {"int8_gemm_tcgen05": "7e9889ec198664ca"}
+NCU_TRAFFIC = {"int8_gemm_tcgen05": (120.57e6 + 102.05e6 + 153.29e6) / 3}
+NCU_TRAFFIC_SOURCE_SHA = {"int8_gemm_tcgen05": "e6de16be0d278602"}
 
 
 def source_sha(rel: str) -> str:
