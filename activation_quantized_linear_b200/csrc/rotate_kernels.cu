@@ -258,12 +258,11 @@ __device__ __forceinline__ void store_codes32_div(int8_t* base, const uint64_t (
 // the product is rounded toward zero to float32 and its last bit forced to one
 // when inexact ("round to odd"); float32 keeps more than two extra bits, so
 // rounding that to bf16 is the correctly rounded result.
-__device__ __forceinline__ uint32_t bf16x2_exact_product(uint64_t s2, uint64_t v) {
+__device__ __forceinline__ uint32_t bf16x2_exact_product(uint64_t s2, uint64_t neg_s2, uint64_t v) {
   const uint64_t p = mulrz2(s2, v);
-  uint32_t lo, hi;
+  const uint64_t e = fma2(neg_s2, v, p);  // exact p - s*v
+  uint32_t lo, hi, e_lo, e_hi;
   unpk(p, lo, hi);
-  const uint64_t e = fma2(s2, v, pku(lo ^ 0x80000000u, hi ^ 0x80000000u));  // exact s*v - p
-  uint32_t e_lo, e_hi;
   unpk(e, e_lo, e_hi);
   // the remainder is +0 exactly when the product is exact (x - x rounds to +0)
   asm("{\n\t.reg .pred q;\n\t"
@@ -278,10 +277,10 @@ __device__ __forceinline__ uint32_t bf16x2_exact_product(uint64_t s2, uint64_t v
 template <int G>
 __device__ __forceinline__ void store_bf16_32(uint16_t* base, const uint64_t (&P)[kPairs], float sn,
                                               uint32_t lane) {
-  const uint64_t s2 = pk(sn, sn);
+  const uint64_t s2 = pk(sn, sn), neg_s2 = pk(-sn, -sn);
   uint32_t w[kPairs];
 #pragma unroll
-  for (int i = 0; i < kPairs; ++i) w[i] = bf16x2_exact_product(s2, P[i]);  // elements 2i, 2i + 1
+  for (int i = 0; i < kPairs; ++i) w[i] = bf16x2_exact_product(s2, neg_s2, P[i]);  // elements 2i, 2i + 1
   if constexpr (G == 256) {
     const uint32_t t = lane & 7;
     uint16_t* grp = base - kVec * t;
@@ -327,45 +326,56 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
 // A warp stages 32 consecutive chunks of kParts 16-byte units each (bf16:
-// 4, int8: 2) in a slot of its own.  Copy j of lane i moves unit j * 32 + i, so
-// each copy instruction reads 512 contiguous bytes; unit u sits at position
-// stage_pos(u), which rotates every row of 8 units by (u >> 3) so that the
-// copies' stores and the lanes' reads of their own units (kParts * lane + k)
-// both fall in distinct banks.
-__device__ __forceinline__ uint32_t stage_pos(uint32_t u) {
-  return (u & ~7u) | ((u + (u >> 3)) & 7u);
+// 4, int8: 2) in a slot of its own.  Copy j of lane i moves unit 32 j + i, so
+// each copy instruction reads 512 contiguous bytes; lane L later reads its
+// units kParts * L + k.  Unit (L, k) sits at position kParts * L + (L >> s) + k,
+// s = log2(8 / kParts): the gaps make both sides conflict-free (8 lanes of a
+// phase hit 8 distinct 16-byte bank groups) and both sides' addresses a
+// per-lane base plus a constant: the copy's position is i + (i >> 3) + 36 j,
+// the read's kParts * L + (L >> s) + k.
+constexpr int kStageUnitsPerWarp = 144;  // positions 0 .. 142
+constexpr int kStageBytesPerWarp = kStageUnitsPerWarp * 16;
+
+__device__ __forceinline__ uint32_t stage_copy_offset(uint32_t lane) {
+  return (lane + (lane >> 3)) * 16;
+}
+template <int kParts>
+__device__ __forceinline__ uint32_t stage_read_offset(uint32_t lane) {
+  return (kParts * lane + (lane >> (kParts == 4 ? 1 : 2))) * 16;
 }
 
-// chunks chunk0 .. chunk0 + 31 of a row whose chunk c starts at
-// base + c * kParts * 16; chunks at or past `nvalid` copy chunk 0 instead
+// Copies j = 0 .. kParts-1 of one lane: 16 bytes from src + 512 j to
+// dst + 576 j, each only when 32 / kParts * j < lim (the unit's chunk exists).
 template <int kParts>
-__device__ __forceinline__ void stage_chunks(uint32_t slot, uint32_t lane, const uint8_t* base,
-                                             int64_t chunk0, int64_t nvalid) {
+__device__ __forceinline__ void stage_copies(uint32_t dst, const uint8_t* src, int lim) {
 #pragma unroll
   for (int j = 0; j < kParts; ++j) {
-    const uint32_t u = j * 32 + lane;
-    const int64_t c = chunk0 + u / kParts;
-    cp_async16(slot + stage_pos(u) * 16,
-               base + ((c < nvalid ? c : 0) * kParts + u % kParts) * 16);
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.lt.s32 p, %2, %3;\n\t"
+        "@p cp.async.cg.shared.global [%0], [%1], 16;\n\t}"
+        ::"r"(dst + 576 * j), "l"(src + 512 * j), "r"((32 / kParts) * j), "r"(lim)
+        : "memory");
   }
   cp_async_commit();
 }
 
 template <int kParts>
-__device__ __forceinline__ void unstage_chunk(uint32_t slot, uint32_t lane, uint4 (&v)[kParts]) {
+__device__ __forceinline__ void unstage_chunk(uint32_t src, uint4 (&v)[kParts]) {
 #pragma unroll
   for (int k = 0; k < kParts; ++k) {
     asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
                  : "=r"(v[k].x), "=r"(v[k].y), "=r"(v[k].z), "=r"(v[k].w)
-                 : "r"(slot + stage_pos(kParts * lane + k) * 16)
+                 : "r"(src + 16 * k)
                  : "memory");
   }
 }
 
-constexpr int kStageBytesPerWarp = 32 * kVec * 2;
-
-template <int G>
-__global__ void __launch_bounds__(1024) rotate_quant_act_hadamard(
+// kWide: CTAs of at most 256 threads (rows up to 8192 elements), compiled
+// for 3 CTAs per SM with room for 85 registers; otherwise teams of up to
+// 1024 threads at 64 registers.
+template <int G, bool kWide>
+__global__ void __launch_bounds__(kWide ? 256 : 1024, kWide ? 3 : 1) rotate_quant_act_hadamard(
     const uint16_t* __restrict__ x, int64_t M, int K, int team_warps, int rows_per_cta,
     int8_t* __restrict__ xq, float* __restrict__ s_tok) {
   extern __shared__ __align__(16) uint8_t smem_all[];
@@ -379,34 +389,35 @@ __global__ void __launch_bounds__(1024) rotate_quant_act_hadamard(
   const int nwarps = blockDim.x >> 5;
   const uint32_t slot = smem_addr(smem_all) + warp * kStageBytesPerWarp;
   const uint32_t xch = smem_addr(smem_all) + nwarps * kStageBytesPerWarp + warp * xch_bytes_per_warp<G>();
-  const int64_t blocks = (M + rows_per_cta - 1) / rows_per_cta;
+  const uint32_t cp_dst = slot + stage_copy_offset(lane);
+  const uint32_t rd_src = slot + stage_read_offset<4>(lane);
+  // copy j of this lane holds part of chunk t0 + 8 j + lane / 4 of the row
+  const int lim = nch - t0 - static_cast<int>(lane >> 2);
+  const uint8_t* xb = reinterpret_cast<const uint8_t*>(x) + (static_cast<int64_t>(t0) * 64 + 16 * lane);
+  const int64_t row_bytes = static_cast<int64_t>(K) * 2;
   constexpr float norm = Norm<G>::value;
 
   // The CTA walks row blocks blockIdx.x, blockIdx.x + gridDim.x, ...; the next
   // block's chunks are copied into shared memory while this one is transformed.
-  // Lanes without a chunk (the row's tail, rows past M) are given chunk 0 of a
-  // valid row instead; whole groups share `ok`, and their maxima are dropped.
+  // Lanes without a chunk (the row's tail, rows past M) copy nothing and
+  // transform stale data; whole groups share `ok`, and their results are dropped.
   const int bar_id = 1 + team, bar_threads = team_warps * 32;
-  int64_t rb = blockIdx.x;
-  if (rb < blocks) {
-    const int64_t r = rb * rows_per_cta + team;
-    stage_chunks<4>(slot, lane, reinterpret_cast<const uint8_t*>(x + (r < M ? r : 0) * K), t0, nch);
-  }
-  for (int it = 0; rb < blocks; rb += gridDim.x, ++it) {
-    const int64_t row = rb * rows_per_cta + team;
-    const bool row_ok = row < M;  // uniform over the team
-    const bool ok = row_ok && t < nch;
+  const int64_t row_step = static_cast<int64_t>(gridDim.x) * rows_per_cta;
+  const int64_t src_step = row_step * row_bytes;
+  int64_t row = static_cast<int64_t>(blockIdx.x) * rows_per_cta + team;
+  const uint8_t* src = xb + row * row_bytes;
+  stage_copies<4>(cp_dst, src, row < M ? lim : 0);
+  for (int it = 0; row - team < M; row += row_step, ++it) {
+    const bool ok = row < M && t < nch;  // row < M is uniform over the team
     uint4 u[4];
     cp_async_wait_all();
     __syncwarp();  // the lanes' copies landed: every lane's units are visible
-    unstage_chunk<4>(slot, lane, u);
+    unstage_chunk<4>(rd_src, u);
     uint64_t P[kPairs];
     widen_bf16_32(u, P);
     __syncwarp();  // every lane has read its units before the slot is refilled
-    if (rb + gridDim.x < blocks) {
-      const int64_t r = (rb + gridDim.x) * rows_per_cta + team;
-      stage_chunks<4>(slot, lane, reinterpret_cast<const uint8_t*>(x + (r < M ? r : 0) * K), t0, nch);
-    }
+    src += src_step;
+    stage_copies<4>(cp_dst, src, row + row_step < M ? lim : 0);
     fwht32<G>(P, xch, lane);
     float amax = warp_max(ok ? absmax32(P) : 0.f);
     if (team_warps > 1) {
@@ -446,19 +457,27 @@ __global__ void __launch_bounds__(256, MODE == kFlatDequant ? 3 : 4) hadamard_fl
   extern __shared__ __align__(16) uint8_t smem_all[];
   const uint32_t lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
-  const uint32_t slot = smem_addr(smem_all) + warp * (kParts * 512);
+  const uint32_t slot = smem_addr(smem_all) + warp * kStageBytesPerWarp;
   const uint32_t xch =
-      smem_addr(smem_all) + (blockDim.x >> 5) * (kParts * 512) + warp * xch_bytes_per_warp<G>();
+      smem_addr(smem_all) + (blockDim.x >> 5) * kStageBytesPerWarp + warp * xch_bytes_per_warp<G>();
+  const uint32_t cp_dst = slot + stage_copy_offset(lane);
+  const uint32_t rd_src = slot + stage_read_offset<kParts>(lane);
   const int64_t blocks = (nchunks + blockDim.x - 1) / blockDim.x;
-  const uint8_t* src = static_cast<const uint8_t*>(in);
+  // copy j of this lane holds part of chunk b * blockDim.x + 32 warp + (32 / kParts) j + lane / kParts
+  const uint8_t* src = static_cast<const uint8_t*>(in) +
+                       (static_cast<int64_t>(warp) * 32 * kParts + lane) * 16;
+  const int64_t lim0 = nchunks - warp * 32 - static_cast<int>(lane / kParts);
+  const int64_t block_bytes = static_cast<int64_t>(blockDim.x) * kParts * 16;
   constexpr float norm = Norm<G>::value;
 
   // Chunk c = b * blockDim.x + thread for blocks b = blockIdx.x, + gridDim.x, ...;
-  // the next block's chunk is copied into shared memory while this one is
-  // transformed.  Lanes past the end copy chunk 0 (whole groups share `ok`)
-  // and are dropped.
+  // the next block's chunks are copied into shared memory while this one is
+  // transformed.  Lanes past the end copy nothing and transform stale data
+  // (whole groups share `ok`); their results are dropped.
   auto stage = [&](int64_t b) {
-    stage_chunks<kParts>(slot, lane, src, b * blockDim.x + warp * 32, nchunks);
+    const int64_t lim = lim0 - b * blockDim.x;
+    stage_copies<kParts>(cp_dst, src + b * block_bytes,
+                         lim > 32 ? 32 : static_cast<int>(lim < 0 ? 0 : lim));
   };
   float mul = 0.f, s = 0.f, run_max = 0.f;
   if constexpr (MODE == kFlatQuant) {
@@ -466,14 +485,14 @@ __global__ void __launch_bounds__(256, MODE == kFlatDequant ? 3 : 4) hadamard_fl
     mul = s > 0.f ? norm * (1.f / s) : 0.f;
   }
   int64_t b = blockIdx.x;
-  if (b < blocks) stage(b);
+  stage(b);
   for (; b < blocks; b += gridDim.x) {
     const int64_t c = b * blockDim.x + threadIdx.x;
     const bool ok = c < nchunks;
     uint4 u[kParts];
     cp_async_wait_all();
     __syncwarp();  // the lanes' copies landed: every lane's units are visible
-    unstage_chunk<kParts>(slot, lane, u);
+    unstage_chunk<kParts>(rd_src, u);
     uint64_t P[kPairs];
     if constexpr (MODE == kFlatDequant) {
       widen_i8_32(u, P);
@@ -481,7 +500,7 @@ __global__ void __launch_bounds__(256, MODE == kFlatDequant ? 3 : 4) hadamard_fl
       widen_bf16_32(u, P);
     }
     __syncwarp();  // every lane has read its units before the slot is refilled
-    if (b + gridDim.x < blocks) stage(b + gridDim.x);
+    stage(b + gridDim.x);
     fwht32<G>(P, xch, lane);
 
     if constexpr (MODE == kFlatAbsmax) {
@@ -644,6 +663,27 @@ cudaError_t allow_smem(Kern kern, size_t bytes) {
                               static_cast<int>(bytes));
 }
 
+template <int G, bool kWide>
+cudaError_t rqa_launch(const uint16_t* x, int64_t M, int K, int team_warps, int rows_per_cta,
+                       int8_t* xq, float* s_tok, cudaStream_t stream) {
+  const int warps = team_warps * rows_per_cta;
+  const size_t smem = static_cast<size_t>(warps) * (kStageBytesPerWarp + xch_bytes_per_warp<G>());
+  cudaError_t e = allow_smem(rotate_quant_act_hadamard<G, kWide>, smem);
+  if (e != cudaSuccess) return e;
+  // enough CTAs to fill every SM (register-limited occupancy), each looping
+  // over row blocks with a one-block-ahead prefetch
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, rotate_quant_act_hadamard<G, kWide>,
+                                                    32 * warps, smem);
+  if (e != cudaSuccess) return e;
+  const int64_t blocks = (M + rows_per_cta - 1) / rows_per_cta;
+  const int64_t cap = static_cast<int64_t>(sm_count()) * (per_sm > 0 ? per_sm : 1);
+  const int64_t grid = blocks < cap ? blocks : cap;
+  rotate_quant_act_hadamard<G, kWide><<<static_cast<unsigned>(grid), 32 * warps, smem, stream>>>(
+      x, M, K, team_warps, rows_per_cta, xq, s_tok);
+  return cudaGetLastError();
+}
+
 template <int G>
 cudaError_t rqa_hadamard(const uint16_t* x, int64_t M, int64_t K, int8_t* xq, float* s_tok,
                          cudaStream_t stream) {
@@ -652,22 +692,10 @@ cudaError_t rqa_hadamard(const uint16_t* x, int64_t M, int64_t K, int8_t* xq, fl
   const int nch = static_cast<int>(K / kVec);
   const int team_warps = (nch + 31) / 32;
   const int rows_per_cta = team_warps >= 8 ? 1 : 8 / team_warps;
-  const int warps = team_warps * rows_per_cta;
-  const size_t smem = static_cast<size_t>(warps) * (kStageBytesPerWarp + xch_bytes_per_warp<G>());
-  cudaError_t e = allow_smem(rotate_quant_act_hadamard<G>, smem);
-  if (e != cudaSuccess) return e;
-  // enough CTAs to fill every SM (register-limited occupancy), each looping
-  // over row blocks with a one-block-ahead prefetch
-  int per_sm = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, rotate_quant_act_hadamard<G>,
-                                                    32 * warps, smem);
-  if (e != cudaSuccess) return e;
-  const int64_t blocks = (M + rows_per_cta - 1) / rows_per_cta;
-  const int64_t cap = static_cast<int64_t>(sm_count()) * (per_sm > 0 ? per_sm : 1);
-  const int64_t grid = blocks < cap ? blocks : cap;
-  rotate_quant_act_hadamard<G><<<static_cast<unsigned>(grid), 32 * warps, smem, stream>>>(
-      x, M, static_cast<int>(K), team_warps, rows_per_cta, xq, s_tok);
-  return cudaGetLastError();
+  if (team_warps * rows_per_cta <= 8) {
+    return rqa_launch<G, true>(x, M, static_cast<int>(K), team_warps, rows_per_cta, xq, s_tok, stream);
+  }
+  return rqa_launch<G, false>(x, M, static_cast<int>(K), team_warps, rows_per_cta, xq, s_tok, stream);
 }
 
 template <int G, int MODE, bool PER_ROW>
@@ -675,8 +703,7 @@ cudaError_t flat_launch(const void* in, int64_t nchunks, int64_t chunks_per_row,
                         const float* scale, void* out, unsigned int* absmax_bits,
                         cudaStream_t stream) {
   constexpr int kThreadsFlat = 256;
-  constexpr int kParts = MODE == kFlatDequant ? 2 : 4;
-  const size_t smem = (kThreadsFlat / 32) * (kParts * 512 + xch_bytes_per_warp<G>());
+  const size_t smem = (kThreadsFlat / 32) * (kStageBytesPerWarp + xch_bytes_per_warp<G>());
   cudaError_t e = allow_smem(hadamard_flat<G, MODE, PER_ROW>, smem);
   if (e != cudaSuccess) return e;
   // one chunk per thread and block; enough CTAs to fill every SM, each looping
