@@ -302,10 +302,10 @@ __device__ __forceinline__ float absmax32(const uint64_t (&P)[kPairs]) {
   return m;
 }
 
+// Max over the warp of non-negative floats (never NaN: the absmax drops NaN
+// inputs); their bit patterns order like their values.
 __device__ __forceinline__ float warp_max(float a) {
-#pragma unroll
-  for (int o = 16; o; o >>= 1) a = fmaxf(a, __shfl_xor_sync(kFull, a, o));
-  return a;
+  return __uint_as_float(__reduce_max_sync(kFull, __float_as_uint(a)));
 }
 
 template <int G>
@@ -371,11 +371,11 @@ __device__ __forceinline__ void unstage_chunk(uint32_t src, uint4 (&v)[kParts]) 
   }
 }
 
-// kWide: CTAs of at most 256 threads (rows up to 8192 elements), compiled
-// for 3 CTAs per SM with room for 85 registers; otherwise teams of up to
-// 1024 threads at 64 registers.
-template <int G, bool kWide>
-__global__ void __launch_bounds__(kWide ? 256 : 1024, kWide ? 3 : 1) rotate_quant_act_hadamard(
+// Register budgets by CTA size: kMaxThreads threads, kMinBlocks CTAs per SM
+// (256, 3) and (384, 2) leave room for 85 registers; (1024, 1) keeps 64, so
+// that teams of up to 512 threads still fit two CTAs per SM.
+template <int G, int kMaxThreads, int kMinBlocks>
+__global__ void __launch_bounds__(kMaxThreads, kMinBlocks) rotate_quant_act_hadamard(
     const uint16_t* __restrict__ x, int64_t M, int K, int team_warps, int rows_per_cta,
     int8_t* __restrict__ xq, float* __restrict__ s_tok) {
   extern __shared__ __align__(16) uint8_t smem_all[];
@@ -425,8 +425,7 @@ __global__ void __launch_bounds__(kWide ? 256 : 1024, kWide ? 3 : 1) rotate_quan
       if (lane == 0) rb_red[warp] = amax;
       // the team's warps only: teams of one CTA run independently
       asm volatile("bar.sync %0, %1;" ::"r"(bar_id), "r"(bar_threads) : "memory");
-      amax = 0.f;
-      for (int k = 0; k < team_warps; ++k) amax = fmaxf(amax, rb_red[team * team_warps + k]);
+      amax = warp_max(static_cast<int>(lane) < team_warps ? rb_red[team * team_warps + lane] : 0.f);
     }
     if (!ok) continue;
     const float sc = (amax * norm) / 127.f;  // s_tok = max |x_rot| / 127
@@ -663,23 +662,23 @@ cudaError_t allow_smem(Kern kern, size_t bytes) {
                               static_cast<int>(bytes));
 }
 
-template <int G, bool kWide>
+template <int G, int kMaxThreads, int kMinBlocks>
 cudaError_t rqa_launch(const uint16_t* x, int64_t M, int K, int team_warps, int rows_per_cta,
                        int8_t* xq, float* s_tok, cudaStream_t stream) {
   const int warps = team_warps * rows_per_cta;
   const size_t smem = static_cast<size_t>(warps) * (kStageBytesPerWarp + xch_bytes_per_warp<G>());
-  cudaError_t e = allow_smem(rotate_quant_act_hadamard<G, kWide>, smem);
+  cudaError_t e = allow_smem(rotate_quant_act_hadamard<G, kMaxThreads, kMinBlocks>, smem);
   if (e != cudaSuccess) return e;
   // enough CTAs to fill every SM (register-limited occupancy), each looping
   // over row blocks with a one-block-ahead prefetch
   int per_sm = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, rotate_quant_act_hadamard<G, kWide>,
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, rotate_quant_act_hadamard<G, kMaxThreads, kMinBlocks>,
                                                     32 * warps, smem);
   if (e != cudaSuccess) return e;
   const int64_t blocks = (M + rows_per_cta - 1) / rows_per_cta;
   const int64_t cap = static_cast<int64_t>(sm_count()) * (per_sm > 0 ? per_sm : 1);
   const int64_t grid = blocks < cap ? blocks : cap;
-  rotate_quant_act_hadamard<G, kWide><<<static_cast<unsigned>(grid), 32 * warps, smem, stream>>>(
+  rotate_quant_act_hadamard<G, kMaxThreads, kMinBlocks><<<static_cast<unsigned>(grid), 32 * warps, smem, stream>>>(
       x, M, K, team_warps, rows_per_cta, xq, s_tok);
   return cudaGetLastError();
 }
@@ -692,10 +691,15 @@ cudaError_t rqa_hadamard(const uint16_t* x, int64_t M, int64_t K, int8_t* xq, fl
   const int nch = static_cast<int>(K / kVec);
   const int team_warps = (nch + 31) / 32;
   const int rows_per_cta = team_warps >= 8 ? 1 : 8 / team_warps;
-  if (team_warps * rows_per_cta <= 8) {
-    return rqa_launch<G, true>(x, M, static_cast<int>(K), team_warps, rows_per_cta, xq, s_tok, stream);
+  const int warps = team_warps * rows_per_cta;
+  const int k = static_cast<int>(K);
+  // 9-10 warps fit three CTAs per SM only at 64 registers; 11-12 fit two
+  // CTAs either way, so they take the larger budget
+  if (warps <= 8) return rqa_launch<G, 256, 3>(x, M, k, team_warps, rows_per_cta, xq, s_tok, stream);
+  if (warps >= 11 && warps <= 12) {
+    return rqa_launch<G, 384, 2>(x, M, k, team_warps, rows_per_cta, xq, s_tok, stream);
   }
-  return rqa_launch<G, false>(x, M, static_cast<int>(K), team_warps, rows_per_cta, xq, s_tok, stream);
+  return rqa_launch<G, 1024, 1>(x, M, k, team_warps, rows_per_cta, xq, s_tok, stream);
 }
 
 template <int G, int MODE, bool PER_ROW>
