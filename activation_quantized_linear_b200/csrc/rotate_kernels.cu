@@ -274,13 +274,28 @@ __device__ __forceinline__ uint32_t bf16x2_exact_product(uint64_t s2, uint64_t n
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
+// Round-to-odd without the remainder: p | 1 on the product rounded toward
+// zero.  Exact whenever no product s * v is itself a bf16 midpoint: v is an
+// integer (|v| <= 127 G < 2^15), so s * v has at least as many significant
+// bits as s's mantissa without its trailing zeros; with fewer than 15
+// trailing zeros that is more than the 9 bits of a midpoint (s normal, so the
+// products stay in the normal range).  p | 1 is then correct whether or not
+// the product was exact, since an exact p is no midpoint.
+__device__ __forceinline__ bool odd_rounding_is_exact(float s) {
+  const uint32_t b = __float_as_uint(s);
+  return (b & 0x7FFFu) != 0 && (b & 0x7F800000u) != 0;
+}
+
+__device__ __forceinline__ uint32_t bf16x2_product_fast(uint64_t s2, uint64_t v) {
+  uint32_t lo, hi;
+  unpk(mulrz2(s2, v), lo, hi);
+  const __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(lo | 1u), __uint_as_float(hi | 1u));
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
 template <int G>
-__device__ __forceinline__ void store_bf16_32(uint16_t* base, const uint64_t (&P)[kPairs], float sn,
-                                              uint32_t lane) {
-  const uint64_t s2 = pk(sn, sn), neg_s2 = pk(-sn, -sn);
-  uint32_t w[kPairs];
-#pragma unroll
-  for (int i = 0; i < kPairs; ++i) w[i] = bf16x2_exact_product(s2, neg_s2, P[i]);  // elements 2i, 2i + 1
+__device__ __forceinline__ void store_bf16_words(uint16_t* base, const uint32_t (&w)[kPairs],
+                                                 uint32_t lane) {
   if constexpr (G == 256) {
     const uint32_t t = lane & 7;
     uint16_t* grp = base - kVec * t;
@@ -293,6 +308,22 @@ __device__ __forceinline__ void store_bf16_32(uint16_t* base, const uint64_t (&P
 #pragma unroll
     for (int j = 0; j < 4; ++j) q[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
   }
+}
+
+template <int G>
+__device__ __forceinline__ void store_bf16_32(uint16_t* base, const uint64_t (&P)[kPairs], float sn,
+                                              uint32_t lane) {
+  const uint64_t s2 = pk(sn, sn);
+  uint32_t w[kPairs];
+  if (odd_rounding_is_exact(sn)) {
+#pragma unroll
+    for (int i = 0; i < kPairs; ++i) w[i] = bf16x2_product_fast(s2, P[i]);  // elements 2i, 2i + 1
+  } else {
+    const uint64_t neg_s2 = pk(-sn, -sn);
+#pragma unroll
+    for (int i = 0; i < kPairs; ++i) w[i] = bf16x2_exact_product(s2, neg_s2, P[i]);
+  }
+  store_bf16_words<G>(base, w, lane);
 }
 
 __device__ __forceinline__ float absmax32(const uint64_t (&P)[kPairs]) {

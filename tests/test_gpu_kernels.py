@@ -255,6 +255,32 @@ def test_dequant_derotate_per_channel_scale(kind):
         assert np.all(np.abs(got - ref) <= bf16_ulp(ref))
 
 
+@pytest.mark.parametrize("G", [16, 256])
+def test_dequant_derotate_short_mantissa_scales(G):
+    """Scales with few significant bits make many products s_w * 2^-k * sum
+    exact, some of them exactly halfway between two bf16 values, where only
+    round-half-to-even is right.  The decode must still round each value once
+    (bit-exact against the oracle), per tensor and per output channel, with
+    long- and short-mantissa channel scales mixed."""
+    N, K = 160, 1024
+    R = workloads.sylvester_rotation(G)
+    rot = cr.Rotation(R)
+    rng = np.random.default_rng(G)
+    Wq = _codes(rng, (N, K))
+    for s_w in (2.0 ** -9, 0.375 * 2.0 ** -6, (65 / 128) * 2.0 ** -8):
+        W_hat = cr.dequant_derotate(torch.from_numpy(Wq).cuda(),
+                                    torch.tensor([s_w], dtype=torch.float32, device="cuda"), rot)
+        ref = oracle.dequant_derotate(Wq, s_w, R)
+        np.testing.assert_array_equal(bf16_bits(W_hat), oracle.bf16_bits(ref))
+    s = (rng.random(N) * 1e-3 + 1e-4).astype(np.float32)
+    s[::3] = 2.0 ** -10
+    s[1::7] = 0.75 * 2.0 ** -9
+    W_hat = cr.dequant_derotate(torch.from_numpy(Wq).cuda(), torch.from_numpy(s).cuda(), rot)
+    ref = oracle.bf16_round(s.astype(np.float64)[:, None]
+                            * oracle.block_rotate(Wq.astype(np.float64), R.astype(np.float64).T))
+    np.testing.assert_array_equal(oracle.as_f64(W_hat.cpu()), ref)
+
+
 # ---------------------------------------------------------------------------
 # the whole int8-compute layer
 # ---------------------------------------------------------------------------
