@@ -310,20 +310,18 @@ __device__ __forceinline__ void store_bf16_words(uint16_t* base, const uint32_t 
   }
 }
 
-template <int G>
-__device__ __forceinline__ void store_bf16_32(uint16_t* base, const uint64_t (&P)[kPairs], float sn,
-                                              uint32_t lane) {
+// bf16 words of the 32 products s * P (pairs 2i, 2i + 1 in w[i]), each rounded once.
+__device__ __forceinline__ void bf16_products32(uint32_t (&w)[kPairs], const uint64_t (&P)[kPairs],
+                                                float sn) {
   const uint64_t s2 = pk(sn, sn);
-  uint32_t w[kPairs];
   if (odd_rounding_is_exact(sn)) {
 #pragma unroll
-    for (int i = 0; i < kPairs; ++i) w[i] = bf16x2_product_fast(s2, P[i]);  // elements 2i, 2i + 1
+    for (int i = 0; i < kPairs; ++i) w[i] = bf16x2_product_fast(s2, P[i]);
   } else {
     const uint64_t neg_s2 = pk(-sn, -sn);
 #pragma unroll
     for (int i = 0; i < kPairs; ++i) w[i] = bf16x2_exact_product(s2, neg_s2, P[i]);
   }
-  store_bf16_words<G>(base, w, lane);
 }
 
 __device__ __forceinline__ float absmax32(const uint64_t (&P)[kPairs]) {
@@ -477,6 +475,13 @@ __global__ void __launch_bounds__(kMaxThreads, kMinBlocks) rotate_quant_act_hada
 // ===========================================================================
 enum FlatMode { kFlatAbsmax = 0, kFlatQuant = 1, kFlatDequant = 2 };
 
+// Per-warp shared memory of the flat kernel besides its staging slot: the
+// G = 256 exchange, or the output slot of the decode at G < 256.
+template <int G, int MODE>
+__host__ __device__ constexpr int flat_aux_bytes() {
+  return G == 256 ? kXchBytesPerWarp : (MODE == kFlatDequant ? kStageBytesPerWarp : 0);
+}
+
 template <int G, int MODE, bool PER_ROW_SCALE>
 __global__ void __launch_bounds__(256, MODE == kFlatDequant ? 3 : 4) hadamard_flat(const void* __restrict__ in, int64_t nchunks,
                                                      int64_t chunks_per_row,
@@ -488,8 +493,9 @@ __global__ void __launch_bounds__(256, MODE == kFlatDequant ? 3 : 4) hadamard_fl
   const uint32_t lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const uint32_t slot = smem_addr(smem_all) + warp * kStageBytesPerWarp;
-  const uint32_t xch =
-      smem_addr(smem_all) + (blockDim.x >> 5) * kStageBytesPerWarp + warp * xch_bytes_per_warp<G>();
+  // G = 256: the butterfly exchange; decode at G < 256: the output slot
+  const uint32_t aux =
+      smem_addr(smem_all) + (blockDim.x >> 5) * kStageBytesPerWarp + warp * flat_aux_bytes<G, MODE>();
   const uint32_t cp_dst = slot + stage_copy_offset(lane);
   const uint32_t rd_src = slot + stage_read_offset<kParts>(lane);
   const int64_t blocks = (nchunks + blockDim.x - 1) / blockDim.x;
@@ -531,7 +537,7 @@ __global__ void __launch_bounds__(256, MODE == kFlatDequant ? 3 : 4) hadamard_fl
     }
     __syncwarp();  // every lane has read its units before the slot is refilled
     stage(b + gridDim.x);
-    fwht32<G>(P, xch, lane);
+    fwht32<G>(P, aux, lane);
 
     if constexpr (MODE == kFlatAbsmax) {
       if (ok) run_max = fmaxf(run_max, absmax32(P));
@@ -545,9 +551,39 @@ __global__ void __launch_bounds__(256, MODE == kFlatDequant ? 3 : 4) hadamard_fl
         }
       }
     } else {
-      if (ok) {
-        const float sw = PER_ROW_SCALE ? scale[c / chunks_per_row] : scale[0];
-        store_bf16_32<G>(static_cast<uint16_t*>(out) + c * kVec, P, sw * norm, lane);
+      const float sw = PER_ROW_SCALE ? scale[(ok ? c : 0) / chunks_per_row] : scale[0];
+      uint32_t w[kPairs];
+      bf16_products32(w, P, sw * norm);
+      if constexpr (G == 256) {
+        if (ok) store_bf16_words<G>(static_cast<uint16_t*>(out) + c * kVec, w, lane);
+      } else {
+        // A lane's 64 output bytes are 4 units of the warp's 2 KB; through the
+        // output slot, store j of lane i writes unit 32 j + i (512 contiguous
+        // bytes per instruction) when its chunk exists.
+        const uint32_t wr = aux + stage_read_offset<4>(lane);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(wr + 16 * k),
+                       "r"(w[4 * k]), "r"(w[4 * k + 1]), "r"(w[4 * k + 2]), "r"(w[4 * k + 3])
+                       : "memory");
+        }
+        __syncwarp();
+        const int64_t chunk0 = b * blockDim.x + warp * 32;
+        const int64_t olim = nchunks - chunk0 - static_cast<int>(lane >> 2);
+        uint8_t* dst = static_cast<uint8_t*>(out) + chunk0 * 64 + lane * 16;
+        const uint32_t rd = aux + stage_copy_offset(lane);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          if (8 * j < olim) {
+            uint4 v;
+            asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                         : "r"(rd + 576 * j)
+                         : "memory");
+            *reinterpret_cast<uint4*>(dst + 512 * j) = v;
+          }
+        }
+        __syncwarp();  // the slot is read out before the next block writes it
       }
     }
   }
@@ -738,7 +774,7 @@ cudaError_t flat_launch(const void* in, int64_t nchunks, int64_t chunks_per_row,
                         const float* scale, void* out, unsigned int* absmax_bits,
                         cudaStream_t stream) {
   constexpr int kThreadsFlat = 256;
-  const size_t smem = (kThreadsFlat / 32) * (kStageBytesPerWarp + xch_bytes_per_warp<G>());
+  const size_t smem = (kThreadsFlat / 32) * (kStageBytesPerWarp + flat_aux_bytes<G, MODE>());
   cudaError_t e = allow_smem(hadamard_flat<G, MODE, PER_ROW>, smem);
   if (e != cudaSuccess) return e;
   // one chunk per thread and block; enough CTAs to fill every SM, each looping
