@@ -109,6 +109,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
+  // the set-up above overlaps the previous kernel of the stream; every global
+  // access below comes after it
+  ptx::grid_dependency_wait();
+  ptx::grid_dependents_launch();
 
   if (threadIdx.x == 0) {
     // ------------------------------------------------------------ producer
@@ -267,13 +271,15 @@ cudaError_t launch_nt(const GemmArgs& a, SkinnyParams p, cudaStream_t stream) {
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = C::kSmem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = splits;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, int8_gemm_skinny<NT>, tmW, tmX, p);
 }
 

@@ -25,6 +25,7 @@
 #include <cstdint>
 
 #include "internal.h"
+#include "sm100_ptx.cuh"
 
 namespace convrot {
 namespace {
@@ -432,6 +433,9 @@ __global__ void __launch_bounds__(kMaxThreads, kMinBlocks) rotate_quant_act_hada
   // transform stale data; whole groups share `ok`, and their results are dropped.
   const int bar_id = 1 + team, bar_threads = team_warps * 32;
   const int64_t row_step = static_cast<int64_t>(gridDim.x) * rows_per_cta;
+  // launched chained to the previous kernel: global memory only after it completes
+  ptx::grid_dependency_wait();
+  ptx::grid_dependents_launch();
   const int64_t src_step = row_step * row_bytes;
   int64_t row = static_cast<int64_t>(blockIdx.x) * rows_per_cta + team;
   const uint8_t* src = xb + row * row_bytes;
@@ -515,6 +519,9 @@ __global__ void __launch_bounds__(256, MODE == kFlatDequant ? 3 : 4) hadamard_fl
     stage_copies<kParts>(cp_dst, src + b * block_bytes,
                          lim > 32 ? 32 : static_cast<int>(lim < 0 ? 0 : lim));
   };
+  // launched chained to the previous kernel: global memory only after it completes
+  ptx::grid_dependency_wait();
+  ptx::grid_dependents_launch();
   float mul = 0.f, s = 0.f, run_max = 0.f;
   if constexpr (MODE == kFlatQuant) {
     s = __uint_as_float(*absmax_bits) / 127.f;
@@ -720,6 +727,25 @@ __global__ void finalize_scales(float* __restrict__ s, int64_t n) {
   if (i < n) s[i] = s[i] / 127.f;
 }
 
+// Launches `kern` chained to the previous kernel of the stream (programmatic
+// dependent launch): it may be scheduled while that kernel drains and waits
+// on the device before touching global memory.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_chained(void (*kern)(KArgs...), int64_t grid, int block, size_t smem,
+                           cudaStream_t stream, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(static_cast<unsigned>(block));
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 // Opts the kernel in to `bytes` of dynamic shared memory (the default limit,
 // 48 KB, counts the kernel's static shared memory too).
 template <typename Kern>
@@ -745,9 +771,8 @@ cudaError_t rqa_launch(const uint16_t* x, int64_t M, int K, int team_warps, int 
   const int64_t blocks = (M + rows_per_cta - 1) / rows_per_cta;
   const int64_t cap = static_cast<int64_t>(sm_count()) * (per_sm > 0 ? per_sm : 1);
   const int64_t grid = blocks < cap ? blocks : cap;
-  rotate_quant_act_hadamard<G, kMaxThreads, kMinBlocks><<<static_cast<unsigned>(grid), 32 * warps, smem, stream>>>(
-      x, M, K, team_warps, rows_per_cta, xq, s_tok);
-  return cudaGetLastError();
+  return launch_chained(rotate_quant_act_hadamard<G, kMaxThreads, kMinBlocks>, grid, 32 * warps, smem,
+                        stream, x, M, K, team_warps, rows_per_cta, xq, s_tok);
 }
 
 template <int G>
@@ -786,9 +811,8 @@ cudaError_t flat_launch(const void* in, int64_t nchunks, int64_t chunks_per_row,
   int64_t grid = (nchunks + kThreadsFlat - 1) / kThreadsFlat;
   if (grid > cap) grid = cap;
   if (grid < 1) grid = 1;
-  hadamard_flat<G, MODE, PER_ROW><<<static_cast<unsigned>(grid), kThreadsFlat, smem, stream>>>(
-      in, nchunks, chunks_per_row, scale, out, absmax_bits);
-  return cudaGetLastError();
+  return launch_chained(hadamard_flat<G, MODE, PER_ROW>, grid, kThreadsFlat, smem, stream, in,
+                        nchunks, chunks_per_row, scale, out, absmax_bits);
 }
 
 template <int G, typename TIn, int MODE>

@@ -10,6 +10,19 @@
 namespace convrot {
 namespace ptx {
 
+// ---------------------------------------------------------------- launch chaining
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialisation may start while the previous kernel of the stream finishes.
+// It must pass grid_dependency_wait() (every earlier grid complete, its memory
+// visible) before it reads or writes global memory; grid_dependents_launch()
+// lets the next such kernel be scheduled early.
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void grid_dependents_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
