@@ -42,8 +42,8 @@ INT8_PER_BF16 = 2.0  # nominal dense int8 : bf16 tensor throughput (4.5 : 2.25 P
 # DRAM bytes per launch from ncu (dram__bytes_read.sum + dram__bytes_write.sum),
 # averaged over the three GEMM launches of one Z-Image step, valid only for the
 # kernel source they were taken on (first 16 hex digits of its sha256).
-NCU_TRAFFIC = {"int8_gemm_tcgen05": (120.57e6 + 102.05e6 + 153.29e6) / 3}
-NCU_TRAFFIC_SOURCE_SHA = {"int8_gemm_tcgen05": "e6de16be0d278602"}
+NCU_TRAFFIC = {"int8_gemm_tcgen05": (121.15e6 + 101.11e6 + 156.34e6) / 3}
+NCU_TRAFFIC_SOURCE_SHA = {"int8_gemm_tcgen05": "2022ccd4d06aee17"}
 
 
 def source_sha(rel: str) -> str:
@@ -80,11 +80,11 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "20"],
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
-        time.sleep(0.3)
+        time.sleep(0.1)
         return self
 
     def __exit__(self, *exc):
@@ -110,13 +110,25 @@ class ClockSampler:
                 os.unlink(self.path)
         if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        def num(v):
+            try:
+                return float(v)
+            except ValueError:
+                return None
+        # samples under load: power draw in the upper half between the lowest
+        # and highest draw seen (the idle samples around the region drop out)
+        power = [num(r[3]) for r in rows]
+        known = [w for w in power if w is not None]
+        cut = (min(known) + max(known)) / 2 if known and max(known) - min(known) > 50 else None
+        loaded = [r for r, w in zip(rows, power) if cut is None or (w is not None and w >= cut)]
+        sm = [num(r[1]) for r in loaded if num(r[1]) is not None]
+        mx = [num(r[2]) for r in rows if num(r[2]) is not None]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v == "Active"})
         return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
-                "samples": len(rows)}
+                "samples": len(rows), "samples_under_load": len(loaded),
+                "max_power_w": max(known) if known else None}
 
 
 # ---------------------------------------------------------------------------
@@ -218,7 +230,7 @@ def run_reference(args, lins):
         "value": value, "unit": "TOPS", "n_gpus": args.gpus, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": 1e3 * statistics.mean(step_s),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": config_dict(args, lins),
+        "data": "synthetic", "config": config_dict(args, lins, gpu=False),
         "cpu_baseline": {"value": value, "unit": "TOPS", "cores": cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0,
@@ -228,14 +240,21 @@ def run_reference(args, lins):
     return 0
 
 
-def config_dict(args, lins):
-    return {
+def config_dict(args, lins, gpu=True):
+    cfg = {
         "workload": args.workload,
         "linears": [f"{l.name}:M{l.M}xK{l.K}->N{l.N}" for l in lins],
         "G": lins[0].G, "rotation": "sylvester-hadamard",
-        "l2": "flushed between timed steps (256 MiB write + 256 MiB read, untimed)",
-        "launch": "each step enqueued behind a 0.2 ms GPU spin, so host launch gaps are not timed",
     }
+    if gpu:
+        cfg.update({
+            "l2": "flushed between timed steps (256 MiB write + 256 MiB read, untimed)",
+            "launch": "each step enqueued behind a 0.2 ms GPU spin, so host launch gaps are not timed",
+            "timing": "step: CUDA events at step start and end only (kernels chained as in use); "
+                      "per-kernel times and the roofline: an extra step after each timed step, "
+                      "with events between kernels",
+        })
+    return cfg
 
 
 # ---------------------------------------------------------------------------
@@ -290,28 +309,40 @@ def run_ours(args, lins):
     def ev():
         return torch.cuda.Event(enable_timing=True)
 
-    def step(record):
+    def step(record=None):
+        """One pass of the hot path; with `record`, events between the kernels."""
         for i, L in enumerate(layers):
-            e0, e1, e2 = record[i]
-            e0.record(stream)
+            if record:
+                record[i][0].record(stream)
             cr.rotate_quant_act(L["x"], rot, xq=L["xq"], s_tok=L["s_tok"])
-            e1.record(stream)
+            if record:
+                record[i][1].record(stream)
             cr.int8_gemm(L["xq"], L["s_tok"], L["Wq"], L["s_w"], L["bias"], out=L["y"])
-            e2.record(stream)
+            if record:
+                record[i][2].record(stream)
 
     # ---------------- warm-up
     for _ in range(args.warmup):
-        step([(ev(), ev(), ev()) for _ in range(n_lin)])
+        step()
     torch.cuda.synchronize()
     cr.check_status()
 
-    # ---------------- timed: int8-compute forward
+    # ---------------- timed: int8-compute forward.  Each timed step is
+    # bracketed by two events only, so consecutive kernels overlap as they do
+    # in use; every timed step is followed by a breakdown step with events
+    # between the kernels (same clocks and power state), whose per-kernel
+    # times give the roofline.
+    steps_ev = [(ev(), ev()) for _ in range(args.steps)]
     recs = [[(ev(), ev(), ev()) for _ in range(n_lin)] for _ in range(args.steps)]
     barrier(world)
     torch.cuda.synchronize()
     with ClockSampler(local) as clocks:
         for k in range(args.steps):
-            flush_l2(k)
+            flush_l2(2 * k)
+            steps_ev[k][0].record(stream)
+            step()
+            steps_ev[k][1].record(stream)
+            flush_l2(2 * k + 1)
             step(recs[k])
         torch.cuda.synchronize()
     barrier(world)
@@ -320,7 +351,7 @@ def run_ours(args, lins):
 
     rqa_ms = np.array([[r[i][0].elapsed_time(r[i][1]) for i in range(n_lin)] for r in recs])
     gemm_ms = np.array([[r[i][1].elapsed_time(r[i][2]) for i in range(n_lin)] for r in recs])
-    step_ms = np.array([r[0][0].elapsed_time(r[-1][2]) for r in recs])
+    step_ms = np.array([e0.elapsed_time(e1) for e0, e1 in steps_ev])
     ops_step = sum(2.0 * L["lin"].M * L["lin"].N * L["lin"].K for L in layers)
     value, total_ms = weak_scaling_throughput(ops_step, args.steps, float(step_ms.sum()), world, dev)
 
@@ -473,7 +504,7 @@ def run_sweep(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="zimage_dit_block",
