@@ -13,6 +13,8 @@ from .convrot_oracle import (  # noqa: F401
     cosine,
     dequant_derotate,
     epilogue,
+    f16_bits,
+    f16_round,
     int8_gemm_acc,
     linear_dense,
     linear_int8,
@@ -20,4 +22,5 @@ from .convrot_oracle import (  # noqa: F401
     quantize_weight,
     rel_l2,
     rotate_quant_act,
+    round16,
 )

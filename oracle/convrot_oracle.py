@@ -38,6 +38,10 @@ Readings where the pages leave a step open (each is a choice, stated once):
   its output row is the bias.
 * epilogue: y = bf16_rn(acc * s_tok * s_w + bias), evaluated in float64 and
   rounded once to bf16.
+* 16-bit formats: the layer runs with BF16 or FP16 activations ([INT8C],
+  opening section and the "Running in FP32" row of its table); in fp16 the
+  inputs are read exactly and every output (decoded weight, layer output) is
+  rounded once to fp16 instead of bf16.
 """
 
 from __future__ import annotations
@@ -69,6 +73,34 @@ def bf16_round(v) -> np.ndarray:
     e = np.maximum(e, -125)               # bf16 normal floor: 2^-126 = 0.5 * 2^-125
     ulp = np.ldexp(1.0, e - 8)            # spacing of 8-significant-bit numbers
     return np.rint(v / ulp) * ulp         # np.rint rounds half to even; exact in fp64
+
+
+def f16_round(v) -> np.ndarray:
+    """Round float64 values to the nearest IEEE fp16 (ties to even), returned as
+    float64.  A single rounding, straight from float64: 11 significant bits,
+    exponent floor of the fp16 normal range (2^-14), so subnormals are
+    multiples of 2^-24; magnitudes that round above 65504 become infinite.
+    """
+    v = np.asarray(v, dtype=np.float64)
+    _, e = np.frexp(v)                    # v = m * 2^e, 0.5 <= |m| < 1
+    e = np.maximum(e, -13)                # fp16 normal floor: 2^-14 = 0.5 * 2^-13
+    ulp = np.ldexp(1.0, e - 11)           # spacing of 11-significant-bit numbers
+    r = np.rint(v / ulp) * ulp
+    return np.where(np.abs(r) > 65504.0, np.copysign(np.inf, v), r)
+
+
+def round16(v, fmt: str) -> np.ndarray:
+    """The 16-bit output rounding of the layer: "bf16" or "f16"."""
+    if fmt == "bf16":
+        return bf16_round(v)
+    if fmt == "f16":
+        return f16_round(v)
+    raise ValueError(fmt)
+
+
+def f16_bits(v) -> np.ndarray:
+    """fp16-representable float64 values -> their uint16 bit patterns."""
+    return np.asarray(v, dtype=np.float64).astype(np.float16).view(np.uint16)
 
 
 def bf16_bits(v) -> np.ndarray:
@@ -126,15 +158,16 @@ def quantize_weight(W, R):
     return quantize_symmetric(W_rot, s_w), s_w
 
 
-def dequant_derotate(Wq, s_w, R) -> np.ndarray:
-    """Default (weight-decode) path: W_hat = bf16(s_w * Wq . B_R^T).
+def dequant_derotate(Wq, s_w, R, fmt: str = "bf16") -> np.ndarray:
+    """Default (weight-decode) path: W_hat = bf16(s_w * Wq . B_R^T) (fp16 with
+    fmt="f16").
 
     [PR194] "Summary": each quantized layer "dequantizes and derotates per
     forward"; the derotation is the product [out, in/G, G] @ [G, G].
-    Returns the bf16 values as float64 [N, K].
+    Returns the 16-bit values as float64 [N, K].
     """
     R = as_f64(R)
-    return bf16_round(np.float64(np.float32(s_w)) * block_rotate(np.asarray(Wq, np.float64), R.T))
+    return round16(np.float64(np.float32(s_w)) * block_rotate(np.asarray(Wq, np.float64), R.T), fmt)
 
 
 def rotate_quant_act(x, R):
@@ -171,29 +204,30 @@ def int8_gemm_acc(xq, Wq) -> np.ndarray:
     return acc.astype(np.int64).astype(np.int32)
 
 
-def epilogue(acc, s_tok, s_w, bias=None) -> np.ndarray:
-    """int8_compute, step 3: y = bf16(acc * s_tok[m] * s_w + bias[n]).
+def epilogue(acc, s_tok, s_w, bias=None, fmt: str = "bf16") -> np.ndarray:
+    """int8_compute, step 3: y = bf16(acc * s_tok[m] * s_w + bias[n]) (fp16 with
+    fmt="f16").
 
     [INT8C] opening section and "Layer / Why" table (outputs are BF16/FP16);
     the bias is the nn.Linear bias the layer replaces ([PR194] "Summary").
-    Returns the bf16 values as float64 [M, N].
+    Returns the 16-bit values as float64 [M, N].
     """
     y = (np.asarray(acc, np.float64)
          * np.asarray(s_tok, np.float32).astype(np.float64)[:, None]
          * np.float64(np.float32(s_w)))
     if bias is not None:
         y = y + as_f64(bias)[None, :]
-    return bf16_round(y)
+    return round16(y, fmt)
 
 
-def linear_int8(x, Wq, s_w, R, bias=None):
+def linear_int8(x, Wq, s_w, R, bias=None, fmt: str = "bf16"):
     """The whole int8_compute forward: rotate+quantize, int8 GEMM, epilogue.
 
     [INT8C] opening section.  Returns (y, xq, s_tok, acc).
     """
     xq, s_tok = rotate_quant_act(x, R)
     acc = int8_gemm_acc(xq, Wq)
-    return epilogue(acc, s_tok, s_w, bias), xq, s_tok, acc
+    return epilogue(acc, s_tok, s_w, bias, fmt), xq, s_tok, acc
 
 
 def linear_dense(x, W, bias=None) -> np.ndarray:

@@ -239,8 +239,34 @@ def check_rotation_helps_outliers(o):
     assert errs["H"] < 0.25 * errs["I"]
 
 
+def check_f16_round(o):
+    """IEEE binary16 rounding from its definition: 11 significant bits, ties to
+    even, subnormals at multiples of 2^-24 below 2^-14, overflow past 65504
+    (the midpoint 65520 and up) to infinity; then against numpy's own float16
+    conversion of float32 values (a library routine); and the two fp16 outputs
+    of the layer (the epilogue and the decode) round the same way."""
+    cases = {
+        1 + 2.0 ** -11: 1.0, 1 + 3 * 2.0 ** -11: 1 + 2.0 ** -9, 2049.0: 2048.0, 2051.0: 2052.0,
+        65504.0: 65504.0, 65519.0: 65504.0, 65520.0: np.inf, -65520.0: -np.inf,
+        2.0 ** -24: 2.0 ** -24, 2.0 ** -25: 0.0, 3 * 2.0 ** -25: 2.0 ** -23,
+        2.0 ** -14 + 2.0 ** -25: 2.0 ** -14, -(2.0 ** -14 + 3 * 2.0 ** -25): -(2.0 ** -14 + 2.0 ** -23),
+    }
+    for v, want in cases.items():
+        assert o.f16_round(np.array([v]))[0] == want, v
+    rng = np.random.default_rng(16)
+    v = (rng.standard_normal(20000) * np.exp2(rng.integers(-30, 17, 20000))).astype(np.float32)
+    np.testing.assert_array_equal(o.f16_round(v.astype(np.float64)),
+                                  v.astype(np.float16).astype(np.float64))
+    acc = np.array([[2049, 4097]], np.int32)
+    np.testing.assert_array_equal(
+        o.epilogue(acc, np.array([1.0], np.float32), 1.0, None, "f16"), [[2048.0, 4096.0]])
+    Wq = np.array([[100, 3, 0, 0]], np.int8)   # H/2 rows: (103, 97, 103, 97) / 2
+    np.testing.assert_array_equal(o.dequant_derotate(Wq, 1.0, H4_HALF, "f16"),
+                                  [[51.5, 48.5, 51.5, 48.5]])
+
+
 CHECKS = [
-    check_worked_example, check_block_rotate_bruteforce, check_block_rotate_direction,
+    check_f16_round, check_worked_example, check_block_rotate_bruteforce, check_block_rotate_direction,
     check_rotation_identity, check_round_trip, check_bf16_round, check_quantize_symmetric,
     check_act_quant_properties, check_zero_token, check_gemm_bruteforce, check_gemm_extremes,
     check_epilogue_closed_forms, check_weight_decode_accuracy, check_layer_accuracy,
@@ -279,8 +305,8 @@ def _mutant(**overrides):
     return m
 
 
-def _bug_skip_derotation(Wq, s_w, R):
-    return real_oracle.bf16_round(np.float64(np.float32(s_w)) * np.asarray(Wq, np.float64))
+def _bug_skip_derotation(Wq, s_w, R, fmt="bf16"):
+    return real_oracle.round16(np.float64(np.float32(s_w)) * np.asarray(Wq, np.float64), fmt)
 
 
 def _bug_transposed_rotation(A, R):
@@ -290,8 +316,8 @@ def _bug_transposed_rotation(A, R):
     return (A.reshape(A.shape[0], -1, G) @ R).reshape(A.shape)
 
 
-def _bug_drop_bias(acc, s_tok, s_w, bias=None):
-    return real_oracle.epilogue(acc, s_tok, s_w, None)
+def _bug_drop_bias(acc, s_tok, s_w, bias=None, fmt="bf16"):
+    return real_oracle.epilogue(acc, s_tok, s_w, None, fmt)
 
 
 def _bug_group_scale(x, R):
@@ -322,6 +348,21 @@ def _bug_bf16_via_fp32(v):
     return torch.from_numpy(np.atleast_1d(f)).to(torch.bfloat16).double().numpy().reshape(np.shape(f))
 
 
+def _bug_f16_ten_bits(v):
+    v = np.asarray(v, np.float64)
+    _, e = np.frexp(v)
+    ulp = np.ldexp(1.0, np.maximum(e, -13) - 10)
+    return np.rint(v / ulp) * ulp
+
+
+def _bug_f16_no_subnormals(v):
+    v = np.asarray(v, np.float64)
+    _, e = np.frexp(v)
+    ulp = np.ldexp(1.0, e - 11)
+    r = np.rint(v / ulp) * ulp
+    return np.where(np.abs(r) > 65504.0, np.copysign(np.inf, v), r)
+
+
 def _bug_scale_255(W, R):
     W_rot = real_oracle.block_rotate(W, R)
     s_w = np.float32(np.max(np.abs(W_rot)) / 255)
@@ -337,6 +378,8 @@ MUTANTS = {
     "truncating_round": dict(quantize_symmetric=_bug_truncating_round),
     "bf16_double_rounding": dict(bf16_round=_bug_bf16_via_fp32),
     "weight_scale_255": dict(quantize_weight=_bug_scale_255),
+    "f16_ten_significant_bits": dict(f16_round=_bug_f16_ten_bits),
+    "f16_without_subnormals": dict(f16_round=_bug_f16_no_subnormals),
 }
 
 

@@ -76,13 +76,14 @@ SEED_X, SEED_X_OUTLIERS, SEED_W, SEED_W_OUTLIERS, SEED_BIAS, SEED_QR = (
     1000, 2000, 3000, 4000, 5000, 6000)
 
 
-def to_bf16(a: np.ndarray) -> torch.Tensor:
-    """fp32 numpy array -> bf16 CPU tensor (round to nearest even)."""
-    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(torch.bfloat16)
+def to_bf16(a: np.ndarray, dtype: torch.dtype = torch.bfloat16) -> torch.Tensor:
+    """fp32 numpy array -> bf16 (or `dtype`, e.g. fp16) CPU tensor (round to nearest even)."""
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(dtype)
 
 
 def make_activation(M: int, K: int, seed: int, n_outliers: int = 4,
-                    outlier_seed: int | None = None, scale: float = 30.0) -> torch.Tensor:
+                    outlier_seed: int | None = None, scale: float = 30.0,
+                    dtype: torch.dtype = torch.bfloat16) -> torch.Tensor:
     """x ~ N(0,1) [M, K] with `n_outliers` input channels multiplied by `scale`."""
     rng = np.random.default_rng(seed)
     x = rng.standard_normal((M, K), dtype=np.float32)
@@ -90,12 +91,12 @@ def make_activation(M: int, K: int, seed: int, n_outliers: int = 4,
         orng = np.random.default_rng(seed + 1 if outlier_seed is None else outlier_seed)
         cols = orng.choice(K, size=min(n_outliers, K), replace=False)
         x[:, cols] *= scale
-    return to_bf16(x)
+    return to_bf16(x, dtype)
 
 
 def make_weight(N: int, K: int, seed: int, outlier_frac: float = 0.01,
                 outlier_seed: int | None = None, std: float = 0.02,
-                scale: float = 10.0) -> torch.Tensor:
+                scale: float = 10.0, dtype: torch.dtype = torch.bfloat16) -> torch.Tensor:
     """W ~ N(0, std) [N, K] with a fraction of its input columns multiplied by `scale`."""
     rng = np.random.default_rng(seed)
     w = rng.standard_normal((N, K), dtype=np.float32) * np.float32(std)
@@ -104,12 +105,12 @@ def make_weight(N: int, K: int, seed: int, outlier_frac: float = 0.01,
         orng = np.random.default_rng(seed + 1 if outlier_seed is None else outlier_seed)
         cols = orng.choice(K, size=n_cols, replace=False)
         w[:, cols] *= np.float32(scale)
-    return to_bf16(w)
+    return to_bf16(w, dtype)
 
 
-def make_bias(N: int, seed: int, std: float = 0.01) -> torch.Tensor:
+def make_bias(N: int, seed: int, std: float = 0.01, dtype: torch.dtype = torch.bfloat16) -> torch.Tensor:
     rng = np.random.default_rng(seed)
-    return to_bf16(rng.standard_normal(N, dtype=np.float32) * np.float32(std))
+    return to_bf16(rng.standard_normal(N, dtype=np.float32) * np.float32(std), dtype)
 
 
 def sylvester_rotation(G: int) -> np.ndarray:
@@ -137,19 +138,22 @@ def qr_rotation(G: int, seed: int = SEED_QR) -> np.ndarray:
 
 @dataclasses.dataclass
 class LayerInputs:
-    x: torch.Tensor        # bf16 [M, K]
-    W: torch.Tensor        # bf16 [N, K]
-    bias: torch.Tensor     # bf16 [N]
+    x: torch.Tensor        # bf16 or fp16 [M, K]
+    W: torch.Tensor        # bf16 or fp16 [N, K]
+    bias: torch.Tensor     # bf16 or fp16 [N]
     R: np.ndarray          # float32 [G, G]
 
 
 def make_layer_inputs(lin: Linear, index: int = 0, rotation: str = "sylvester",
-                      M: int | None = None) -> LayerInputs:
-    """All inputs of one linear, drawn from the seeds of workload `index`."""
+                      M: int | None = None, dtype: torch.dtype = torch.bfloat16) -> LayerInputs:
+    """All inputs of one linear, drawn from the seeds of workload `index`, as
+    bf16 (or `dtype`, e.g. fp16) tensors."""
     m = lin.M if M is None else M
-    x = make_activation(m, lin.K, SEED_X + index, lin.n_outliers, SEED_X_OUTLIERS + index)
-    W = make_weight(lin.N, lin.K, SEED_W + index, outlier_seed=SEED_W_OUTLIERS + index)
-    b = make_bias(lin.N, SEED_BIAS + index)
+    x = make_activation(m, lin.K, SEED_X + index, lin.n_outliers, SEED_X_OUTLIERS + index,
+                        dtype=dtype)
+    W = make_weight(lin.N, lin.K, SEED_W + index, outlier_seed=SEED_W_OUTLIERS + index,
+                    dtype=dtype)
+    b = make_bias(lin.N, SEED_BIAS + index, dtype=dtype)
     if rotation == "sylvester":
         R = sylvester_rotation(lin.G)
     elif rotation == "qr":
