@@ -74,6 +74,11 @@ def _load() -> ctypes.CDLL:
         "convrot_linear_int8_noalloc": ([vp, i64, i64, i64, vp, vp, vp, i64, vp, vp, vp], i32),
         "convrot_noalloc_scratch_bytes": ([], sz),
         "convrot_check_status": ([vp], i32),
+        "convrot_quantize_weight_f16": ([vp, i64, i64, vp, vp, vp, vp], i32),
+        "convrot_dequant_derotate_f16": ([vp, vp, i64, i64, i64, vp, vp, vp], i32),
+        "convrot_rotate_quant_act_f16": ([vp, i64, i64, vp, vp, vp, vp], i32),
+        "convrot_int8_gemm_f16": ([vp, vp, vp, vp, i64, vp, i64, i64, i64, vp, vp], i32),
+        "convrot_linear_int8_f16": ([vp, i64, i64, i64, vp, vp, vp, i64, vp, vp, vp, sz, vp], i32),
     }
     for name, (args, res) in sigs.items():
         fn = getattr(lib, name)
@@ -109,6 +114,23 @@ def _need(t: torch.Tensor, name: str, dtype: torch.dtype, ndim: int) -> None:
         raise ValueError(f"{name} must be a CUDA tensor")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
+
+
+FLOAT16 = (torch.bfloat16, torch.float16)
+
+
+def _need16(t: torch.Tensor, name: str, ndim: int) -> None:
+    """A bf16 or fp16 tensor (the layer's two activation formats)."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype not in FLOAT16:
+        raise TypeError(f"{name} must be bfloat16 or float16, got {t.dtype}")
+    _need(t, name, t.dtype, ndim)
+
+
+def _fn(name: str, dtype: torch.dtype):
+    """The C entry point for a 16-bit float format: name (bf16) or name_f16."""
+    return getattr(_lib, name + ("_f16" if dtype == torch.float16 else ""))
 
 
 def device_supported(device: int = 0) -> bool:
@@ -161,55 +183,63 @@ class Rotation:
 
 def quantize_weight(W: torch.Tensor, rot: Rotation, Wq: torch.Tensor | None = None,
                     s_w: torch.Tensor | None = None):
-    """W [N, K] bf16 -> (Wq [N, K] int8, s_w [1] float32)."""
-    _need(W, "W", torch.bfloat16, 2)
+    """W [N, K] bf16 or fp16 -> (Wq [N, K] int8, s_w [1] float32)."""
+    _need16(W, "W", 2)
     N, K = W.shape
     Wq = torch.empty((N, K), dtype=torch.int8, device=W.device) if Wq is None else Wq
     s_w = torch.empty(1, dtype=torch.float32, device=W.device) if s_w is None else s_w
-    _check(_lib.convrot_quantize_weight(_ptr(W), N, K, rot.handle, _ptr(Wq), _ptr(s_w), _stream()))
+    _check(_fn("convrot_quantize_weight", W.dtype)(_ptr(W), N, K, rot.handle, _ptr(Wq), _ptr(s_w),
+                                                    _stream()))
     return Wq, s_w
 
 
 def dequant_derotate(Wq: torch.Tensor, s_w: torch.Tensor, rot: Rotation,
-                     out: torch.Tensor | None = None) -> torch.Tensor:
-    """Wq [N, K] int8, s_w [1] or [N] float32 -> W_hat [N, K] bf16."""
+                     out: torch.Tensor | None = None,
+                     dtype: torch.dtype = torch.bfloat16) -> torch.Tensor:
+    """Wq [N, K] int8, s_w [1] or [N] float32 -> W_hat [N, K] in `dtype` (bf16 or
+    fp16; the dtype of `out` when given)."""
     _need(Wq, "Wq", torch.int8, 2)
     _need(s_w, "s_w", torch.float32, 1)
     N, K = Wq.shape
-    out = torch.empty((N, K), dtype=torch.bfloat16, device=Wq.device) if out is None else out
-    _check(_lib.convrot_dequant_derotate(_ptr(Wq), _ptr(s_w), s_w.numel(), N, K, rot.handle,
-                                         _ptr(out), _stream()))
+    out = torch.empty((N, K), dtype=dtype, device=Wq.device) if out is None else out
+    _need16(out, "out", 2)
+    _check(_fn("convrot_dequant_derotate", out.dtype)(_ptr(Wq), _ptr(s_w), s_w.numel(), N, K,
+                                                       rot.handle, _ptr(out), _stream()))
     return out
 
 
 def rotate_quant_act(x: torch.Tensor, rot: Rotation, xq: torch.Tensor | None = None,
                      s_tok: torch.Tensor | None = None):
-    """x [M, K] bf16 -> (xq [M, K] int8, s_tok [M] float32)."""
-    _need(x, "x", torch.bfloat16, 2)
+    """x [M, K] bf16 or fp16 -> (xq [M, K] int8, s_tok [M] float32)."""
+    _need16(x, "x", 2)
     M, K = x.shape
     xq = torch.empty((M, K), dtype=torch.int8, device=x.device) if xq is None else xq
     s_tok = torch.empty(M, dtype=torch.float32, device=x.device) if s_tok is None else s_tok
-    _check(_lib.convrot_rotate_quant_act(_ptr(x), M, K, rot.handle, _ptr(xq), _ptr(s_tok),
-                                         _stream()))
+    _check(_fn("convrot_rotate_quant_act", x.dtype)(_ptr(x), M, K, rot.handle, _ptr(xq),
+                                                     _ptr(s_tok), _stream()))
     return xq, s_tok
 
 
 def int8_gemm(xq: torch.Tensor, s_tok: torch.Tensor, Wq: torch.Tensor, s_w: torch.Tensor,
-              bias: torch.Tensor | None = None, out: torch.Tensor | None = None) -> torch.Tensor:
-    """y = bf16(xq . Wq^T * s_tok[:, None] * s_w + bias)."""
+              bias: torch.Tensor | None = None, out: torch.Tensor | None = None,
+              dtype: torch.dtype = torch.bfloat16) -> torch.Tensor:
+    """y = f16(xq . Wq^T * s_tok[:, None] * s_w + bias) in `dtype` (bf16 or fp16;
+    the dtype of `out` when given); bias, if any, in the same dtype."""
     _need(xq, "xq", torch.int8, 2)
     _need(Wq, "Wq", torch.int8, 2)
     _need(s_tok, "s_tok", torch.float32, 1)
     _need(s_w, "s_w", torch.float32, 1)
-    if bias is not None:
-        _need(bias, "bias", torch.bfloat16, 1)
     M, K = xq.shape
     N = Wq.shape[0]
     if Wq.shape[1] != K:
         raise ValueError("xq and Wq disagree on K")
-    out = torch.empty((M, N), dtype=torch.bfloat16, device=xq.device) if out is None else out
-    _check(_lib.convrot_int8_gemm(_ptr(xq), _ptr(s_tok), _ptr(Wq), _ptr(s_w), s_w.numel(),
-                                  _ptr(bias), M, N, K, _ptr(out), _stream()))
+    out = torch.empty((M, N), dtype=dtype, device=xq.device) if out is None else out
+    _need16(out, "out", 2)
+    if bias is not None:
+        _need(bias, "bias", out.dtype, 1)
+    _check(_fn("convrot_int8_gemm", out.dtype)(_ptr(xq), _ptr(s_tok), _ptr(Wq), _ptr(s_w),
+                                                s_w.numel(), _ptr(bias), M, N, K, _ptr(out),
+                                                _stream()))
     return out
 
 
@@ -233,21 +263,23 @@ def workspace_bytes(M: int, N: int, K: int) -> int:
 def linear_int8(x: torch.Tensor, Wq: torch.Tensor, s_w: torch.Tensor, rot: Rotation,
                 bias: torch.Tensor | None = None, out: torch.Tensor | None = None,
                 workspace: torch.Tensor | None = None) -> torch.Tensor:
-    """The int8-compute forward: rotate+quantize x per token, int8 GEMM, rescale."""
-    _need(x, "x", torch.bfloat16, 2)
+    """The int8-compute forward: rotate+quantize x per token, int8 GEMM, rescale.
+    x, bias and the output share one 16-bit float format (bf16 or fp16)."""
+    _need16(x, "x", 2)
     _need(Wq, "Wq", torch.int8, 2)
     _need(s_w, "s_w", torch.float32, 1)
     if bias is not None:
-        _need(bias, "bias", torch.bfloat16, 1)
+        _need(bias, "bias", x.dtype, 1)
     M, K = x.shape
     N = Wq.shape[0]
     need = workspace_bytes(M, N, K)
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=x.device)
-    out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device) if out is None else out
-    _check(_lib.convrot_linear_int8(_ptr(x), M, K, N, rot.handle, _ptr(Wq), _ptr(s_w), s_w.numel(),
-                                    _ptr(bias), _ptr(out), _ptr(workspace), workspace.numel(),
-                                    _stream()))
+    out = torch.empty((M, N), dtype=x.dtype, device=x.device) if out is None else out
+    _need(out, "out", x.dtype, 2)
+    _check(_fn("convrot_linear_int8", x.dtype)(_ptr(x), M, K, N, rot.handle, _ptr(Wq), _ptr(s_w),
+                                                s_w.numel(), _ptr(bias), _ptr(out),
+                                                _ptr(workspace), workspace.numel(), _stream()))
     return out
 
 
@@ -283,12 +315,14 @@ def check_status(stream: torch.cuda.Stream | None = None) -> None:
 class ConvRotLinear:
     """A ConvRot int8_tensorwise linear: int8 weight, per-tensor scale, rotation R.
 
-    `forward` runs the int8-compute path; `decode_weight` the default path's
-    weight decode (dequantize + derotate to bf16)."""
+    `forward` runs the int8-compute path in the input's format (bf16 or fp16;
+    the bias, if any, must match it); `decode_weight` the default path's weight
+    decode (dequantize + derotate) to W's format unless `dtype` says otherwise."""
 
     def __init__(self, W: torch.Tensor, R, bias: torch.Tensor | None = None):
         self.rotation = R if isinstance(R, Rotation) else Rotation(R)
         self.Wq, self.s_w = quantize_weight(W, self.rotation)
+        self.dtype = W.dtype
         self.bias = bias
         self._ws = None
 
@@ -300,8 +334,10 @@ class ConvRotLinear:
     def in_features(self) -> int:
         return self.Wq.shape[1]
 
-    def decode_weight(self, out: torch.Tensor | None = None) -> torch.Tensor:
-        return dequant_derotate(self.Wq, self.s_w, self.rotation, out=out)
+    def decode_weight(self, out: torch.Tensor | None = None,
+                      dtype: torch.dtype | None = None) -> torch.Tensor:
+        return dequant_derotate(self.Wq, self.s_w, self.rotation, out=out,
+                                dtype=dtype or self.dtype)
 
     def forward(self, x: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
         M = x.shape[0]

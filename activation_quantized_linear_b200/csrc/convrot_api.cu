@@ -226,9 +226,9 @@ convrot_status convrot_rotation_info(convrot_rotation_t R, int* G, int* is_sylve
   return CONVROT_OK;
 }
 
-convrot_status convrot_quantize_weight(const convrot_bf16* W, int64_t N, int64_t K,
-                                       convrot_rotation_t R, int8_t* Wq, float* s_w,
-                                       convrot_stream_t stream) {
+static convrot_status quantize_weight_impl(const uint16_t* W, bool f16, int64_t N, int64_t K,
+                                           convrot_rotation_t R, int8_t* Wq, float* s_w,
+                                           convrot_stream_t stream) {
   CHECK_PTR(W);
   CHECK_PTR(Wq);
   if (s_w == nullptr) return fail(CONVROT_ERR_INVALID_ARG, "s_w is NULL");
@@ -239,13 +239,25 @@ convrot_status convrot_quantize_weight(const convrot_bf16* W, int64_t N, int64_t
   if (s != CONVROT_OK) return s;
   s = check_rotation(R);
   if (s != CONVROT_OK) return s;
-  return launched(convrot::launch_quantize_weight(R, W, N, K, Wq, s_w, as_stream(stream)),
+  return launched(convrot::launch_quantize_weight(R, W, f16, N, K, Wq, s_w, as_stream(stream)),
                   "quantize_weight launch");
 }
 
-convrot_status convrot_dequant_derotate(const int8_t* Wq, const float* s_w, int64_t s_w_len,
-                                        int64_t N, int64_t K, convrot_rotation_t R,
-                                        convrot_bf16* W_hat, convrot_stream_t stream) {
+convrot_status convrot_quantize_weight(const convrot_bf16* W, int64_t N, int64_t K,
+                                       convrot_rotation_t R, int8_t* Wq, float* s_w,
+                                       convrot_stream_t stream) {
+  return quantize_weight_impl(W, false, N, K, R, Wq, s_w, stream);
+}
+
+convrot_status convrot_quantize_weight_f16(const convrot_f16* W, int64_t N, int64_t K,
+                                           convrot_rotation_t R, int8_t* Wq, float* s_w,
+                                           convrot_stream_t stream) {
+  return quantize_weight_impl(W, true, N, K, R, Wq, s_w, stream);
+}
+
+static convrot_status dequant_derotate_impl(const int8_t* Wq, const float* s_w, int64_t s_w_len,
+                                            int64_t N, int64_t K, convrot_rotation_t R,
+                                            uint16_t* W_hat, bool f16, convrot_stream_t stream) {
   CHECK_PTR(Wq);
   CHECK_PTR(W_hat);
   if (s_w == nullptr) return fail(CONVROT_ERR_INVALID_ARG, "s_w is NULL");
@@ -260,13 +272,25 @@ convrot_status convrot_dequant_derotate(const int8_t* Wq, const float* s_w, int6
   s = check_rotation(R);
   if (s != CONVROT_OK) return s;
   return launched(
-      convrot::launch_dequant_derotate(R, Wq, s_w, s_w_len, N, K, W_hat, as_stream(stream)),
+      convrot::launch_dequant_derotate(R, Wq, s_w, s_w_len, N, K, W_hat, f16, as_stream(stream)),
       "dequant_derotate launch");
 }
 
-convrot_status convrot_rotate_quant_act(const convrot_bf16* x, int64_t M, int64_t K,
-                                        convrot_rotation_t R, int8_t* xq, float* s_tok,
-                                        convrot_stream_t stream) {
+convrot_status convrot_dequant_derotate(const int8_t* Wq, const float* s_w, int64_t s_w_len,
+                                        int64_t N, int64_t K, convrot_rotation_t R,
+                                        convrot_bf16* W_hat, convrot_stream_t stream) {
+  return dequant_derotate_impl(Wq, s_w, s_w_len, N, K, R, W_hat, false, stream);
+}
+
+convrot_status convrot_dequant_derotate_f16(const int8_t* Wq, const float* s_w, int64_t s_w_len,
+                                            int64_t N, int64_t K, convrot_rotation_t R,
+                                            convrot_f16* W_hat, convrot_stream_t stream) {
+  return dequant_derotate_impl(Wq, s_w, s_w_len, N, K, R, W_hat, true, stream);
+}
+
+static convrot_status rotate_quant_act_impl(const uint16_t* x, bool f16, int64_t M, int64_t K,
+                                            convrot_rotation_t R, int8_t* xq, float* s_tok,
+                                            convrot_stream_t stream) {
   if (M < 0 || M >= kMaxDim) return fail(CONVROT_ERR_INVALID_ARG, "M=%lld out of range", (long long)M);
   if (R == nullptr) return fail(CONVROT_ERR_INVALID_ARG, "rotation handle is NULL");
   convrot_status s = check_rotation_shape(R, K);
@@ -281,13 +305,25 @@ convrot_status convrot_rotate_quant_act(const convrot_bf16* x, int64_t M, int64_
   if (s_tok == nullptr) return fail(CONVROT_ERR_INVALID_ARG, "s_tok is NULL");
   s = check_rotation(R);
   if (s != CONVROT_OK) return s;
-  return launched(convrot::launch_rotate_quant_act(R, x, M, K, xq, s_tok, as_stream(stream)),
+  return launched(convrot::launch_rotate_quant_act(R, x, f16, M, K, xq, s_tok, as_stream(stream)),
                   "rotate_quant_act launch");
 }
 
+convrot_status convrot_rotate_quant_act(const convrot_bf16* x, int64_t M, int64_t K,
+                                        convrot_rotation_t R, int8_t* xq, float* s_tok,
+                                        convrot_stream_t stream) {
+  return rotate_quant_act_impl(x, false, M, K, R, xq, s_tok, stream);
+}
+
+convrot_status convrot_rotate_quant_act_f16(const convrot_f16* x, int64_t M, int64_t K,
+                                            convrot_rotation_t R, int8_t* xq, float* s_tok,
+                                            convrot_stream_t stream) {
+  return rotate_quant_act_impl(x, true, M, K, R, xq, s_tok, stream);
+}
+
 static convrot_status gemm_common(const int8_t* xq, const float* s_tok, const int8_t* Wq,
-                                  const float* s_w, int64_t s_w_len, const convrot_bf16* bias,
-                                  int64_t M, int64_t N, int64_t K, void* out, bool s32,
+                                  const float* s_w, int64_t s_w_len, const uint16_t* bias,
+                                  int64_t M, int64_t N, int64_t K, void* out, bool s32, bool f16,
                                   convrot_stream_t stream) {
   convrot_status s = check_gemm_shape(M, N, K);
   if (s != CONVROT_OK) return s;
@@ -324,6 +360,7 @@ static convrot_status gemm_common(const int8_t* xq, const float* s_tok, const in
   a.N = N;
   a.K = K;
   a.out_s32 = s32;
+  a.out_f16 = f16 && !s32;
   cudaError_t e = convrot::launch_int8_gemm(a, as_stream(stream));
   if (e == cudaErrorInvalidValue) {
     return fail(CONVROT_ERR_CUDA, "int8_gemm: TMA descriptor encoding failed");
@@ -335,12 +372,19 @@ convrot_status convrot_int8_gemm(const int8_t* xq, const float* s_tok, const int
                                  const float* s_w, int64_t s_w_len, const convrot_bf16* bias,
                                  int64_t M, int64_t N, int64_t K, convrot_bf16* y,
                                  convrot_stream_t stream) {
-  return gemm_common(xq, s_tok, Wq, s_w, s_w_len, bias, M, N, K, y, false, stream);
+  return gemm_common(xq, s_tok, Wq, s_w, s_w_len, bias, M, N, K, y, false, false, stream);
+}
+
+convrot_status convrot_int8_gemm_f16(const int8_t* xq, const float* s_tok, const int8_t* Wq,
+                                     const float* s_w, int64_t s_w_len, const convrot_f16* bias,
+                                     int64_t M, int64_t N, int64_t K, convrot_f16* y,
+                                     convrot_stream_t stream) {
+  return gemm_common(xq, s_tok, Wq, s_w, s_w_len, bias, M, N, K, y, false, true, stream);
 }
 
 convrot_status convrot_int8_gemm_s32(const int8_t* xq, const int8_t* Wq, int64_t M, int64_t N,
                                      int64_t K, int32_t* acc, convrot_stream_t stream) {
-  return gemm_common(xq, nullptr, Wq, nullptr, 1, nullptr, M, N, K, acc, true, stream);
+  return gemm_common(xq, nullptr, Wq, nullptr, 1, nullptr, M, N, K, acc, true, false, stream);
 }
 
 size_t convrot_workspace_bytes(int op, int64_t M, int64_t N, int64_t K) {
@@ -350,10 +394,11 @@ size_t convrot_workspace_bytes(int op, int64_t M, int64_t N, int64_t K) {
          align256(sizeof(float) * static_cast<size_t>(M));
 }
 
-convrot_status convrot_linear_int8(const convrot_bf16* x, int64_t M, int64_t K, int64_t N,
-                                   convrot_rotation_t R, const int8_t* Wq, const float* s_w,
-                                   int64_t s_w_len, const convrot_bf16* bias, convrot_bf16* y,
-                                   void* ws, size_t ws_bytes, convrot_stream_t stream) {
+static convrot_status linear_int8_impl(const uint16_t* x, bool f16, int64_t M, int64_t K,
+                                       int64_t N, convrot_rotation_t R, const int8_t* Wq,
+                                       const float* s_w, int64_t s_w_len, const uint16_t* bias,
+                                       uint16_t* y, void* ws, size_t ws_bytes,
+                                       convrot_stream_t stream) {
   convrot_status s = check_gemm_shape(M, N, K);
   if (s != CONVROT_OK) return s;
   if (R == nullptr) return fail(CONVROT_ERR_INVALID_ARG, "rotation handle is NULL");
@@ -374,9 +419,23 @@ convrot_status convrot_linear_int8(const convrot_bf16* x, int64_t M, int64_t K, 
   int8_t* xq = static_cast<int8_t*>(ws);
   float* s_tok = reinterpret_cast<float*>(static_cast<char*>(ws) +
                                           align256(static_cast<size_t>(M) * static_cast<size_t>(K)));
-  s = convrot_rotate_quant_act(x, M, K, R, xq, s_tok, stream);
+  s = rotate_quant_act_impl(x, f16, M, K, R, xq, s_tok, stream);
   if (s != CONVROT_OK) return s;
-  return convrot_int8_gemm(xq, s_tok, Wq, s_w, s_w_len, bias, M, N, K, y, stream);
+  return gemm_common(xq, s_tok, Wq, s_w, s_w_len, bias, M, N, K, y, false, f16, stream);
+}
+
+convrot_status convrot_linear_int8(const convrot_bf16* x, int64_t M, int64_t K, int64_t N,
+                                   convrot_rotation_t R, const int8_t* Wq, const float* s_w,
+                                   int64_t s_w_len, const convrot_bf16* bias, convrot_bf16* y,
+                                   void* ws, size_t ws_bytes, convrot_stream_t stream) {
+  return linear_int8_impl(x, false, M, K, N, R, Wq, s_w, s_w_len, bias, y, ws, ws_bytes, stream);
+}
+
+convrot_status convrot_linear_int8_f16(const convrot_f16* x, int64_t M, int64_t K, int64_t N,
+                                       convrot_rotation_t R, const int8_t* Wq, const float* s_w,
+                                       int64_t s_w_len, const convrot_f16* bias, convrot_f16* y,
+                                       void* ws, size_t ws_bytes, convrot_stream_t stream) {
+  return linear_int8_impl(x, true, M, K, N, R, Wq, s_w, s_w_len, bias, y, ws, ws_bytes, stream);
 }
 
 convrot_status convrot_check_status(convrot_stream_t stream) {

@@ -25,6 +25,7 @@
 // issuing work, drains what it issued and frees its TMEM before returning.
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -76,6 +77,7 @@ struct Params {
   int group_m;
   int per_channel_scale;
   int out_s32;
+  int out_f16;           // y and bias fp16 (else bf16)
   unsigned int* status;  // device status word (bit 0: a wait ran out)
 };
 
@@ -113,9 +115,15 @@ __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity) {
   return ptx::mbar_wait(bar, parity, ptx::globaltimer_ns() + kWaitNs);
 }
 
-__device__ __forceinline__ void store_bf16_row32(uint16_t* dst, const uint32_t (&r)[32], float scale,
-                                                 const float* s_w_row, const uint16_t* bias,
-                                                 int valid) {
+// 32 outputs of one row: y = f16(float(acc) * scale [* s_w_row] + bias), in bf16
+// or fp16 (f16), rounded once from the fp32 FMA.
+__device__ __forceinline__ float widen16(uint16_t v, bool f16) {
+  return f16 ? __half2float(__ushort_as_half(v)) : __uint_as_float(static_cast<uint32_t>(v) << 16);
+}
+
+__device__ __forceinline__ void store_row32(uint16_t* dst, const uint32_t (&r)[32], float scale,
+                                            const float* s_w_row, const uint16_t* bias, int valid,
+                                            bool f16) {
   uint32_t w[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
@@ -125,13 +133,18 @@ __device__ __forceinline__ void store_bf16_row32(uint16_t* dst, const uint32_t (
     const float sh = s_w_row ? scale * s_w_row[2 * i + 1] : scale;
     float bl = 0.f, bh = 0.f;
     if (bias) {
-      bl = __uint_as_float(static_cast<uint32_t>(bias[2 * i]) << 16);
-      bh = __uint_as_float(static_cast<uint32_t>(bias[2 * i + 1]) << 16);
+      bl = widen16(bias[2 * i], f16);
+      bh = widen16(bias[2 * i + 1], f16);
     }
     lo = fmaf(lo, sl, bl);
     hi = fmaf(hi, sh, bh);
-    const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
-    w[i] = *reinterpret_cast<const uint32_t*>(&h);
+    if (f16) {
+      const __half2 h = __floats2half2_rn(lo, hi);
+      w[i] = *reinterpret_cast<const uint32_t*>(&h);
+    } else {
+      const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+      w[i] = *reinterpret_cast<const uint32_t*>(&h);
+    }
   }
   uint4* q = reinterpret_cast<uint4*>(dst);
   q[0] = make_uint4(w[0], w[1], w[2], w[3]);
@@ -340,9 +353,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (p.out_s32) {
             store_s32_row32(static_cast<int32_t*>(p.out) + m * p.N + n0, r, valid);
           } else {
-            store_bf16_row32(static_cast<uint16_t*>(p.out) + m * p.N + n0, r, scale,
-                             p.per_channel_scale ? p.s_w + n0 : nullptr,
-                             p.bias ? p.bias + n0 : nullptr, valid);
+            store_row32(static_cast<uint16_t*>(p.out) + m * p.N + n0, r, scale,
+                        p.per_channel_scale ? p.s_w + n0 : nullptr, p.bias ? p.bias + n0 : nullptr,
+                        valid, p.out_f16 != 0);
           }
         }
       }
@@ -436,6 +449,7 @@ cudaError_t launch_int8_gemm(const GemmArgs& a, cudaStream_t stream) {
   p.n_tiles = static_cast<int>((a.N + BN - 1) / BN);
   p.per_channel_scale = a.s_w_len > 1 ? 1 : 0;
   p.out_s32 = a.out_s32 ? 1 : 0;
+  p.out_f16 = a.out_f16 ? 1 : 0;
   // few tokens: the weight-streaming swap-AB kernel; otherwise CTA pairs
   // (256-row tiles) once there is more than one 128-row block of tokens
   if (a.M <= BM) return launch_int8_gemm_skinny(a, stream);

@@ -12,6 +12,7 @@
 // scratch.  Same warp roles and bounded waits as the main GEMM.
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -39,6 +40,7 @@ struct SkinnyParams {
   int splits;        // cluster size S
   int per_channel_scale;
   int out_s32;
+  int out_f16;  // y and bias fp16 (else bf16)
   unsigned int* status;
 };
 
@@ -218,8 +220,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int64_t n = static_cast<int64_t>(block) * kRows + rr;
       if (n >= p.N) continue;
       const float sw = p.out_s32 ? 0.f : (p.per_channel_scale ? p.s_w[n] : p.s_w[0]);
-      const float bn =
-          (!p.out_s32 && p.bias) ? __uint_as_float(static_cast<uint32_t>(p.bias[n]) << 16) : 0.f;
+      float bn = 0.f;
+      if (!p.out_s32 && p.bias) {
+        bn = p.out_f16 ? __half2float(__ushort_as_half(p.bias[n]))
+                       : __uint_as_float(static_cast<uint32_t>(p.bias[n]) << 16);
+      }
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int64_t m = m4 + j;
@@ -228,8 +233,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           static_cast<int32_t*>(p.out)[m * p.N + n] = acc[j];
         } else {
           const float y = fmaf(__int2float_rn(acc[j]), p.s_tok[m] * sw, bn);
-          const __nv_bfloat16 h = __float2bfloat16_rn(y);
-          static_cast<uint16_t*>(p.out)[m * p.N + n] = *reinterpret_cast<const uint16_t*>(&h);
+          uint16_t bits;
+          if (p.out_f16) {
+            bits = __half_as_ushort(__float2half_rn(y));
+          } else {
+            const __nv_bfloat16 h = __float2bfloat16_rn(y);
+            bits = *reinterpret_cast<const uint16_t*>(&h);
+          }
+          static_cast<uint16_t*>(p.out)[m * p.N + n] = bits;
         }
       }
     }
@@ -298,6 +309,7 @@ cudaError_t launch_int8_gemm_skinny(const GemmArgs& a, cudaStream_t stream) {
   p.num_kb = static_cast<int>((a.K + kBK - 1) / kBK);
   p.per_channel_scale = a.s_w_len > 1 ? 1 : 0;
   p.out_s32 = a.out_s32 ? 1 : 0;
+  p.out_f16 = a.out_f16 ? 1 : 0;
   if (a.M <= 16) return launch_nt<16>(a, p, stream);
   if (a.M <= 32) return launch_nt<32>(a, p, stream);
   if (a.M <= 64) return launch_nt<64>(a, p, stream);

@@ -21,30 +21,36 @@ namespace convrot {
 // Each launcher enqueues on `stream` and returns the launch error (cudaSuccess
 // when the kernels were enqueued).  Arguments are validated by the caller.
 
-// x [M, K] bf16 -> xq [M, K] int8, s_tok [M] f32 (per-token scale).
-cudaError_t launch_rotate_quant_act(const convrot_rotation_s* R, const uint16_t* x, int64_t M,
-                                    int64_t K, int8_t* xq, float* s_tok, cudaStream_t stream);
+// x [M, K] bf16 (f16 = false) or fp16 -> xq [M, K] int8, s_tok [M] f32
+// (per-token scale).
+cudaError_t launch_rotate_quant_act(const convrot_rotation_s* R, const uint16_t* x, bool f16,
+                                    int64_t M, int64_t K, int8_t* xq, float* s_tok,
+                                    cudaStream_t stream);
 
-// Wq [N, K] int8 -> W_hat [N, K] bf16, scale s_w[0] (s_w_len == 1) or s_w[n].
+// Wq [N, K] int8 -> W_hat [N, K] bf16 (f16 = false) or fp16, scale s_w[0]
+// (s_w_len == 1) or s_w[n].
 cudaError_t launch_dequant_derotate(const convrot_rotation_s* R, const int8_t* Wq,
                                     const float* s_w, int64_t s_w_len, int64_t N, int64_t K,
-                                    uint16_t* W_hat, cudaStream_t stream);
+                                    uint16_t* W_hat, bool f16, cudaStream_t stream);
 
-// W [N, K] bf16 -> Wq [N, K] int8, s_w[0] (one per-tensor scale).
-cudaError_t launch_quantize_weight(const convrot_rotation_s* R, const uint16_t* W, int64_t N,
-                                   int64_t K, int8_t* Wq, float* s_w, cudaStream_t stream);
+// W [N, K] bf16 (f16 = false) or fp16 -> Wq [N, K] int8, s_w[0] (one
+// per-tensor scale).
+cudaError_t launch_quantize_weight(const convrot_rotation_s* R, const uint16_t* W, bool f16,
+                                   int64_t N, int64_t K, int8_t* Wq, float* s_w,
+                                   cudaStream_t stream);
 
 // ------------------------------------------------------------------ GEMM
 struct GemmArgs {
   const int8_t* A;       // xq [M, K]
   const int8_t* B;       // Wq [N, K]
-  const float* s_tok;    // [M]          (bf16 output only)
-  const float* s_w;      // [1] or [N]   (bf16 output only)
+  const float* s_tok;    // [M]          (16-bit float output only)
+  const float* s_w;      // [1] or [N]   (16-bit float output only)
   int64_t s_w_len;
-  const uint16_t* bias;  // [N] or null
-  void* out;             // bf16 y [M, N] or int32 acc [M, N]
+  const uint16_t* bias;  // [N] or null, in the output's format
+  void* out;             // y [M, N] bf16 / fp16, or int32 acc [M, N]
   int64_t M, N, K;
   bool out_s32;
+  bool out_f16;          // y and bias are fp16 (else bf16)
 };
 
 // Encodes the TMA descriptors and launches the tcgen05 GEMM.  Returns

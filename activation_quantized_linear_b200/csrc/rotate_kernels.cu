@@ -20,6 +20,7 @@
 //     (bf16 or int8) and R (float32) are exact in float64, so each output is
 //     the exact value up to one float64 rounding per term.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -109,6 +110,29 @@ __device__ __forceinline__ void widen_bf16_32(const uint4 (&u)[4], uint64_t (&P)
     for (int k = 0; k < 4; ++k) {
       P[4 * j + k] = pku(w[k] << 16, w[k] & 0xffff0000u);
     }
+  }
+}
+
+// raw fp16 words -> P[i] = (p[2i], p[2i + 1]) as floats (exact).
+__device__ __forceinline__ void widen_f16_32(const uint4 (&u)[4], uint64_t (&P)[kPairs]) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t w[4] = {u[j].x, u[j].y, u[j].z, u[j].w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[k]));
+      P[4 * j + k] = pk(f.x, f.y);
+    }
+  }
+}
+
+// 16-bit float input: bf16 (kF16 = false) or fp16 (kF16 = true).
+template <bool kF16>
+__device__ __forceinline__ void widen16_32(const uint4 (&u)[4], uint64_t (&P)[kPairs]) {
+  if constexpr (kF16) {
+    widen_f16_32(u, P);
+  } else {
+    widen_bf16_32(u, P);
   }
 }
 
@@ -255,14 +279,16 @@ __device__ __forceinline__ void store_codes32_div(int8_t* base, const uint64_t (
   store_code_bytes<G>(base, R, lane);
 }
 
-// bf16 pair of the exact products s * v, each rounded once to nearest-even:
-// the product is rounded toward zero to float32 and its last bit forced to one
-// when inexact ("round to odd"); float32 keeps more than two extra bits, so
-// rounding that to bf16 is the correctly rounded result.
-__device__ __forceinline__ uint32_t bf16x2_exact_product(uint64_t s2, uint64_t neg_s2, uint64_t v) {
+// The exact products s * v of a pair, each rounded once to nearest-even into a
+// 16-bit float: the product is rounded toward zero to float32 and its last
+// bit forced to one when inexact ("round to odd"); float32 keeps at least two
+// bits more than bf16 and fp16 (normal or subnormal results alike), so
+// rounding that to the 16-bit format is the correctly rounded result.
+__device__ __forceinline__ void odd_product2(uint64_t s2, uint64_t neg_s2, uint64_t v, uint32_t& lo,
+                                             uint32_t& hi) {
   const uint64_t p = mulrz2(s2, v);
   const uint64_t e = fma2(neg_s2, v, p);  // exact p - s*v
-  uint32_t lo, hi, e_lo, e_hi;
+  uint32_t e_lo, e_hi;
   unpk(p, lo, hi);
   unpk(e, e_lo, e_hi);
   // the remainder is +0 exactly when the product is exact (x - x rounds to +0)
@@ -271,31 +297,59 @@ __device__ __forceinline__ uint32_t bf16x2_exact_product(uint64_t s2, uint64_t n
       "setp.ne.b32 q, %3, 0;\n\t@q or.b32 %1, %1, 1;\n\t}"
       : "+r"(lo), "+r"(hi)
       : "r"(e_lo), "r"(e_hi));
-  const __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(lo), __uint_as_float(hi));
-  return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-// Round-to-odd without the remainder: p | 1 on the product rounded toward
-// zero.  Exact whenever no product s * v is itself a bf16 midpoint: v is an
-// integer (|v| <= 127 G < 2^15), so s * v has at least as many significant
-// bits as s's mantissa without its trailing zeros; with fewer than 15
-// trailing zeros that is more than the 9 bits of a midpoint (s normal, so the
-// products stay in the normal range).  p | 1 is then correct whether or not
-// the product was exact, since an exact p is no midpoint.
+// Round-to-odd without the remainder (bf16 output): p | 1 on the product
+// rounded toward zero.  Exact whenever no product s * v is itself a bf16
+// midpoint: v is an integer (|v| <= 127 G < 2^15), so s * v has at least as
+// many significant bits as s's mantissa without its trailing zeros; with fewer
+// than 15 trailing zeros that is more than the 9 bits of a midpoint (s normal,
+// so the products stay in bf16's normal range).  p | 1 is then correct whether
+// or not the product was exact, since an exact p is no midpoint.  (fp16 output
+// has no such shortcut: its subnormal midpoints sit at fixed multiples of
+// 2^-25, which exact products can hit.)
 __device__ __forceinline__ bool odd_rounding_is_exact(float s) {
   const uint32_t b = __float_as_uint(s);
   return (b & 0x7FFFu) != 0 && (b & 0x7F800000u) != 0;
 }
 
-__device__ __forceinline__ uint32_t bf16x2_product_fast(uint64_t s2, uint64_t v) {
-  uint32_t lo, hi;
-  unpk(mulrz2(s2, v), lo, hi);
-  const __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(lo | 1u), __uint_as_float(hi | 1u));
-  return *reinterpret_cast<const uint32_t*>(&h);
+template <bool kF16>
+__device__ __forceinline__ uint32_t pack16x2(uint32_t lo, uint32_t hi) {
+  if constexpr (kF16) {
+    const __half2 h = __floats2half2_rn(__uint_as_float(lo), __uint_as_float(hi));
+    return *reinterpret_cast<const uint32_t*>(&h);
+  } else {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(lo), __uint_as_float(hi));
+    return *reinterpret_cast<const uint32_t*>(&h);
+  }
+}
+
+// 16-bit words of the 32 products s * P (pairs 2i, 2i + 1 in w[i]), each
+// rounded once: bf16 (kF16 = false) or fp16.
+template <bool kF16>
+__device__ __forceinline__ void products16_32(uint32_t (&w)[kPairs], const uint64_t (&P)[kPairs],
+                                              float sn) {
+  const uint64_t s2 = pk(sn, sn);
+  if (!kF16 && odd_rounding_is_exact(sn)) {
+#pragma unroll
+    for (int i = 0; i < kPairs; ++i) {
+      uint32_t lo, hi;
+      unpk(mulrz2(s2, P[i]), lo, hi);
+      w[i] = pack16x2<false>(lo | 1u, hi | 1u);
+    }
+  } else {
+    const uint64_t neg_s2 = pk(-sn, -sn);
+#pragma unroll
+    for (int i = 0; i < kPairs; ++i) {
+      uint32_t lo, hi;
+      odd_product2(s2, neg_s2, P[i], lo, hi);
+      w[i] = pack16x2<kF16>(lo, hi);
+    }
+  }
 }
 
 template <int G>
-__device__ __forceinline__ void store_bf16_words(uint16_t* base, const uint32_t (&w)[kPairs],
+__device__ __forceinline__ void store_words16(uint16_t* base, const uint32_t (&w)[kPairs],
                                                  uint32_t lane) {
   if constexpr (G == 256) {
     const uint32_t t = lane & 7;
@@ -308,20 +362,6 @@ __device__ __forceinline__ void store_bf16_words(uint16_t* base, const uint32_t 
     uint4* q = reinterpret_cast<uint4*>(base);
 #pragma unroll
     for (int j = 0; j < 4; ++j) q[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
-  }
-}
-
-// bf16 words of the 32 products s * P (pairs 2i, 2i + 1 in w[i]), each rounded once.
-__device__ __forceinline__ void bf16_products32(uint32_t (&w)[kPairs], const uint64_t (&P)[kPairs],
-                                                float sn) {
-  const uint64_t s2 = pk(sn, sn);
-  if (odd_rounding_is_exact(sn)) {
-#pragma unroll
-    for (int i = 0; i < kPairs; ++i) w[i] = bf16x2_product_fast(s2, P[i]);
-  } else {
-    const uint64_t neg_s2 = pk(-sn, -sn);
-#pragma unroll
-    for (int i = 0; i < kPairs; ++i) w[i] = bf16x2_exact_product(s2, neg_s2, P[i]);
   }
 }
 
@@ -348,10 +388,7 @@ __host__ __device__ constexpr int xch_bytes_per_warp() {
 // 32-element chunk per lane, all loads issued before any arithmetic.  The
 // token's rotated row stays in registers between the absmax and the pack.
 // ===========================================================================
-// Per-lane 16-byte asynchronous copies global -> shared (bypassing L1).
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
+// cp.async groups: commit the copies issued so far, wait for all of them.
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
@@ -404,7 +441,7 @@ __device__ __forceinline__ void unstage_chunk(uint32_t src, uint4 (&v)[kParts]) 
 // Register budgets by CTA size: kMaxThreads threads, kMinBlocks CTAs per SM
 // (256, 3) and (384, 2) leave room for 85 registers; (1024, 1) keeps 64, so
 // that teams of up to 512 threads still fit two CTAs per SM.
-template <int G, int kMaxThreads, int kMinBlocks>
+template <int G, int kMaxThreads, int kMinBlocks, bool kF16>
 __global__ void __launch_bounds__(kMaxThreads, kMinBlocks) rotate_quant_act_hadamard(
     const uint16_t* __restrict__ x, int64_t M, int K, int team_warps, int rows_per_cta,
     int8_t* __restrict__ xq, float* __restrict__ s_tok) {
@@ -447,7 +484,7 @@ __global__ void __launch_bounds__(kMaxThreads, kMinBlocks) rotate_quant_act_hada
     __syncwarp();  // the lanes' copies landed: every lane's units are visible
     unstage_chunk<4>(rd_src, u);
     uint64_t P[kPairs];
-    widen_bf16_32(u, P);
+    widen16_32<kF16>(u, P);
     __syncwarp();  // every lane has read its units before the slot is refilled
     src += src_step;
     stage_copies<4>(cp_dst, src, row + row_step < M ? lim : 0);
@@ -486,7 +523,8 @@ __host__ __device__ constexpr int flat_aux_bytes() {
   return G == 256 ? kXchBytesPerWarp : (MODE == kFlatDequant ? kStageBytesPerWarp : 0);
 }
 
-template <int G, int MODE, bool PER_ROW_SCALE>
+// kF16: the 16-bit float format of W (absmax / quant) or of W_hat (decode).
+template <int G, int MODE, bool PER_ROW_SCALE, bool kF16>
 __global__ void __launch_bounds__(256, MODE == kFlatDequant ? 3 : 4) hadamard_flat(const void* __restrict__ in, int64_t nchunks,
                                                      int64_t chunks_per_row,
                                                      const float* __restrict__ scale,
@@ -540,7 +578,7 @@ __global__ void __launch_bounds__(256, MODE == kFlatDequant ? 3 : 4) hadamard_fl
     if constexpr (MODE == kFlatDequant) {
       widen_i8_32(u, P);
     } else {
-      widen_bf16_32(u, P);
+      widen16_32<kF16>(u, P);
     }
     __syncwarp();  // every lane has read its units before the slot is refilled
     stage(b + gridDim.x);
@@ -560,9 +598,9 @@ __global__ void __launch_bounds__(256, MODE == kFlatDequant ? 3 : 4) hadamard_fl
     } else {
       const float sw = PER_ROW_SCALE ? scale[(ok ? c : 0) / chunks_per_row] : scale[0];
       uint32_t w[kPairs];
-      bf16_products32(w, P, sw * norm);
+      products16_32<kF16>(w, P, sw * norm);
       if constexpr (G == 256) {
-        if (ok) store_bf16_words<G>(static_cast<uint16_t*>(out) + c * kVec, w, lane);
+        if (ok) store_words16<G>(static_cast<uint16_t*>(out) + c * kVec, w, lane);
       } else {
         // A lane's 64 output bytes are 4 units of the warp's 2 KB; through the
         // output slot, store j of lane i writes unit 32 j + i (512 contiguous
@@ -620,7 +658,8 @@ enum DenseMode {
   kDenseDequant = 4,      // bf16 = RN(s_w * value)
 };
 
-template <int G, typename TIn, int MODE>
+// kF16: the 16-bit float format of a uint16_t input, and of the decoded output.
+template <int G, typename TIn, int MODE, bool kF16>
 __global__ void __launch_bounds__(256) dense_rotate(const TIn* __restrict__ in, int64_t group_rows,
                                                     int64_t groups_per_token,
                                                     const float* __restrict__ Rm,
@@ -648,7 +687,8 @@ __global__ void __launch_bounds__(256) dense_rotate(const TIn* __restrict__ in, 
     if (r < group_rows) {
       const TIn raw = in[r * G + (i % G)];
       if constexpr (sizeof(TIn) == 2) {
-        val = __uint_as_float(static_cast<uint32_t>(raw) << 16);
+        val = kF16 ? __half2float(__ushort_as_half(raw))
+                   : __uint_as_float(static_cast<uint32_t>(raw) << 16);
       } else {
         val = static_cast<float>(raw);
       }
@@ -713,8 +753,13 @@ __global__ void __launch_bounds__(256) dense_rotate(const TIn* __restrict__ in, 
         uint16_t* o = static_cast<uint16_t*>(out) + r * G;
 #pragma unroll
         for (int b = 0; b < CPT; ++b) {
-          const __nv_bfloat16 h = __double2bfloat16(static_cast<double>(sw) * acc[a][b]);
-          o[tx + b * TC] = *reinterpret_cast<const uint16_t*>(&h);
+          const double v = static_cast<double>(sw) * acc[a][b];
+          if constexpr (kF16) {
+            o[tx + b * TC] = __half_as_ushort(__double2half(v));
+          } else {
+            const __nv_bfloat16 h = __double2bfloat16(v);
+            o[tx + b * TC] = *reinterpret_cast<const uint16_t*>(&h);
+          }
         }
       }
     }
@@ -755,27 +800,27 @@ cudaError_t allow_smem(Kern kern, size_t bytes) {
                               static_cast<int>(bytes));
 }
 
-template <int G, int kMaxThreads, int kMinBlocks>
+template <int G, int kMaxThreads, int kMinBlocks, bool kF16>
 cudaError_t rqa_launch(const uint16_t* x, int64_t M, int K, int team_warps, int rows_per_cta,
                        int8_t* xq, float* s_tok, cudaStream_t stream) {
   const int warps = team_warps * rows_per_cta;
   const size_t smem = static_cast<size_t>(warps) * (kStageBytesPerWarp + xch_bytes_per_warp<G>());
-  cudaError_t e = allow_smem(rotate_quant_act_hadamard<G, kMaxThreads, kMinBlocks>, smem);
+  cudaError_t e = allow_smem(rotate_quant_act_hadamard<G, kMaxThreads, kMinBlocks, kF16>, smem);
   if (e != cudaSuccess) return e;
   // enough CTAs to fill every SM (register-limited occupancy), each looping
   // over row blocks with a one-block-ahead prefetch
   int per_sm = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, rotate_quant_act_hadamard<G, kMaxThreads, kMinBlocks>,
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, rotate_quant_act_hadamard<G, kMaxThreads, kMinBlocks, kF16>,
                                                     32 * warps, smem);
   if (e != cudaSuccess) return e;
   const int64_t blocks = (M + rows_per_cta - 1) / rows_per_cta;
   const int64_t cap = static_cast<int64_t>(sm_count()) * (per_sm > 0 ? per_sm : 1);
   const int64_t grid = blocks < cap ? blocks : cap;
-  return launch_chained(rotate_quant_act_hadamard<G, kMaxThreads, kMinBlocks>, grid, 32 * warps, smem,
+  return launch_chained(rotate_quant_act_hadamard<G, kMaxThreads, kMinBlocks, kF16>, grid, 32 * warps, smem,
                         stream, x, M, K, team_warps, rows_per_cta, xq, s_tok);
 }
 
-template <int G>
+template <int G, bool kF16>
 cudaError_t rqa_hadamard(const uint16_t* x, int64_t M, int64_t K, int8_t* xq, float* s_tok,
                          cudaStream_t stream) {
   // A token's row is held by a team of ceil(K / 1024) warps, one 32-element
@@ -787,42 +832,44 @@ cudaError_t rqa_hadamard(const uint16_t* x, int64_t M, int64_t K, int8_t* xq, fl
   const int k = static_cast<int>(K);
   // 9-10 warps fit three CTAs per SM only at 64 registers; 11-12 fit two
   // CTAs either way, so they take the larger budget
-  if (warps <= 8) return rqa_launch<G, 256, 3>(x, M, k, team_warps, rows_per_cta, xq, s_tok, stream);
-  if (warps >= 11 && warps <= 12) {
-    return rqa_launch<G, 384, 2>(x, M, k, team_warps, rows_per_cta, xq, s_tok, stream);
+  if (warps <= 8) {
+    return rqa_launch<G, 256, 3, kF16>(x, M, k, team_warps, rows_per_cta, xq, s_tok, stream);
   }
-  return rqa_launch<G, 1024, 1>(x, M, k, team_warps, rows_per_cta, xq, s_tok, stream);
+  if (warps >= 11 && warps <= 12) {
+    return rqa_launch<G, 384, 2, kF16>(x, M, k, team_warps, rows_per_cta, xq, s_tok, stream);
+  }
+  return rqa_launch<G, 1024, 1, kF16>(x, M, k, team_warps, rows_per_cta, xq, s_tok, stream);
 }
 
-template <int G, int MODE, bool PER_ROW>
+template <int G, int MODE, bool PER_ROW, bool kF16>
 cudaError_t flat_launch(const void* in, int64_t nchunks, int64_t chunks_per_row,
                         const float* scale, void* out, unsigned int* absmax_bits,
                         cudaStream_t stream) {
   constexpr int kThreadsFlat = 256;
   const size_t smem = (kThreadsFlat / 32) * (kStageBytesPerWarp + flat_aux_bytes<G, MODE>());
-  cudaError_t e = allow_smem(hadamard_flat<G, MODE, PER_ROW>, smem);
+  cudaError_t e = allow_smem(hadamard_flat<G, MODE, PER_ROW, kF16>, smem);
   if (e != cudaSuccess) return e;
   // one chunk per thread and block; enough CTAs to fill every SM, each looping
   int per_sm = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, hadamard_flat<G, MODE, PER_ROW>,
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, hadamard_flat<G, MODE, PER_ROW, kF16>,
                                                     kThreadsFlat, smem);
   if (e != cudaSuccess) return e;
   const int64_t cap = static_cast<int64_t>(sm_count()) * (per_sm > 0 ? per_sm : 1);
   int64_t grid = (nchunks + kThreadsFlat - 1) / kThreadsFlat;
   if (grid > cap) grid = cap;
   if (grid < 1) grid = 1;
-  return launch_chained(hadamard_flat<G, MODE, PER_ROW>, grid, kThreadsFlat, smem, stream, in,
+  return launch_chained(hadamard_flat<G, MODE, PER_ROW, kF16>, grid, kThreadsFlat, smem, stream, in,
                         nchunks, chunks_per_row, scale, out, absmax_bits);
 }
 
-template <int G, typename TIn, int MODE>
+template <int G, typename TIn, int MODE, bool kF16>
 cudaError_t dense_launch(const TIn* in, int64_t group_rows, int64_t groups_per_token,
                          const float* Rm, const float* scale, int64_t scale_len, void* out,
                          unsigned int* absmax_bits, cudaStream_t stream) {
   constexpr int TMR = 8192 / G;
   constexpr int KC = G < 32 ? G : 32;
   const size_t smem = sizeof(float) * (TMR * G + KC * G);
-  auto kern = dense_rotate<G, TIn, MODE>;
+  auto kern = dense_rotate<G, TIn, MODE, kF16>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
@@ -830,6 +877,12 @@ cudaError_t dense_launch(const TIn* in, int64_t group_rows, int64_t groups_per_t
   kern<<<static_cast<unsigned>(grid), 256, smem, stream>>>(in, group_rows, groups_per_token, Rm,
                                                            scale, scale_len, out, absmax_bits);
   return cudaGetLastError();
+}
+
+// Calls f(std::integral_constant<bool, f16>{}).
+template <typename F>
+cudaError_t by_format(bool f16, F&& f) {
+  return f16 ? f(std::true_type{}) : f(std::false_type{});
 }
 
 template <typename F>
@@ -845,25 +898,31 @@ cudaError_t by_group_size(int G, F&& f) {
 
 }  // namespace
 
-cudaError_t launch_rotate_quant_act(const convrot_rotation_s* R, const uint16_t* x, int64_t M,
-                                    int64_t K, int8_t* xq, float* s_tok, cudaStream_t stream) {
+cudaError_t launch_rotate_quant_act(const convrot_rotation_s* R, const uint16_t* x, bool f16,
+                                    int64_t M, int64_t K, int8_t* xq, float* s_tok,
+                                    cudaStream_t stream) {
   if (M == 0) return cudaSuccess;
   if (R->is_sylvester) {
-    return by_group_size(R->G, [&](auto g) {
-      return rqa_hadamard<decltype(g)::value>(x, M, K, xq, s_tok, stream);
+    return by_format(f16, [&](auto fmt) {
+      return by_group_size(R->G, [&](auto g) {
+        return rqa_hadamard<decltype(g)::value, decltype(fmt)::value>(x, M, K, xq, s_tok, stream);
+      });
     });
   }
   unsigned int* amax = reinterpret_cast<unsigned int*>(s_tok);
   cudaError_t e = cudaMemsetAsync(amax, 0, sizeof(float) * M, stream);
   if (e != cudaSuccess) return e;
   const int64_t gpt = K / R->G;
-  e = by_group_size(R->G, [&](auto g) {
-    constexpr int Gv = decltype(g)::value;
-    cudaError_t r = dense_launch<Gv, uint16_t, kDenseAbsmaxRow>(x, M * gpt, gpt, R->R_dev, nullptr,
-                                                                0, nullptr, amax, stream);
-    if (r != cudaSuccess) return r;
-    return dense_launch<Gv, uint16_t, kDenseQuantRow>(x, M * gpt, gpt, R->R_dev, nullptr, 0, xq,
-                                                      amax, stream);
+  e = by_format(f16, [&](auto fmt) {
+    constexpr bool F = decltype(fmt)::value;
+    return by_group_size(R->G, [&](auto g) {
+      constexpr int Gv = decltype(g)::value;
+      cudaError_t r = dense_launch<Gv, uint16_t, kDenseAbsmaxRow, F>(
+          x, M * gpt, gpt, R->R_dev, nullptr, 0, nullptr, amax, stream);
+      if (r != cudaSuccess) return r;
+      return dense_launch<Gv, uint16_t, kDenseQuantRow, F>(x, M * gpt, gpt, R->R_dev, nullptr, 0,
+                                                           xq, amax, stream);
+    });
   });
   if (e != cudaSuccess) return e;
   finalize_scales<<<static_cast<unsigned>((M + 255) / 256), 256, 0, stream>>>(s_tok, M);
@@ -872,51 +931,59 @@ cudaError_t launch_rotate_quant_act(const convrot_rotation_s* R, const uint16_t*
 
 cudaError_t launch_dequant_derotate(const convrot_rotation_s* R, const int8_t* Wq,
                                     const float* s_w, int64_t s_w_len, int64_t N, int64_t K,
-                                    uint16_t* W_hat, cudaStream_t stream) {
-  if (R->is_sylvester) {
-    const int64_t nchunks = N * K / kVec;
+                                    uint16_t* W_hat, bool f16, cudaStream_t stream) {
+  return by_format(f16, [&](auto fmt) {
+    constexpr bool F = decltype(fmt)::value;
+    if (R->is_sylvester) {
+      const int64_t nchunks = N * K / kVec;
+      return by_group_size(R->G, [&](auto g) {
+        constexpr int Gv = decltype(g)::value;
+        if (s_w_len == 1) {
+          return flat_launch<Gv, kFlatDequant, false, F>(Wq, nchunks, K / kVec, s_w, W_hat,
+                                                         nullptr, stream);
+        }
+        return flat_launch<Gv, kFlatDequant, true, F>(Wq, nchunks, K / kVec, s_w, W_hat, nullptr,
+                                                      stream);
+      });
+    }
+    const int64_t gpt = K / R->G;
     return by_group_size(R->G, [&](auto g) {
-      constexpr int Gv = decltype(g)::value;
-      if (s_w_len == 1) {
-        return flat_launch<Gv, kFlatDequant, false>(Wq, nchunks, K / kVec, s_w, W_hat, nullptr,
-                                                    stream);
-      }
-      return flat_launch<Gv, kFlatDequant, true>(Wq, nchunks, K / kVec, s_w, W_hat, nullptr,
-                                                 stream);
+      return dense_launch<decltype(g)::value, int8_t, kDenseDequant, F>(
+          Wq, N * gpt, gpt, R->Rt_dev, s_w, s_w_len, W_hat, nullptr, stream);
     });
-  }
-  const int64_t gpt = K / R->G;
-  return by_group_size(R->G, [&](auto g) {
-    return dense_launch<decltype(g)::value, int8_t, kDenseDequant>(
-        Wq, N * gpt, gpt, R->Rt_dev, s_w, s_w_len, W_hat, nullptr, stream);
   });
 }
 
-cudaError_t launch_quantize_weight(const convrot_rotation_s* R, const uint16_t* W, int64_t N,
-                                   int64_t K, int8_t* Wq, float* s_w, cudaStream_t stream) {
+cudaError_t launch_quantize_weight(const convrot_rotation_s* R, const uint16_t* W, bool f16,
+                                   int64_t N, int64_t K, int8_t* Wq, float* s_w,
+                                   cudaStream_t stream) {
   unsigned int* amax = reinterpret_cast<unsigned int*>(s_w);
   cudaError_t e = cudaMemsetAsync(amax, 0, sizeof(float), stream);
   if (e != cudaSuccess) return e;
-  if (R->is_sylvester) {
-    const int64_t nchunks = N * K / kVec;
-    e = by_group_size(R->G, [&](auto g) {
-      constexpr int Gv = decltype(g)::value;
-      cudaError_t r = flat_launch<Gv, kFlatAbsmax, false>(W, nchunks, K / kVec, nullptr, nullptr,
-                                                          amax, stream);
-      if (r != cudaSuccess) return r;
-      return flat_launch<Gv, kFlatQuant, false>(W, nchunks, K / kVec, nullptr, Wq, amax, stream);
-    });
-  } else {
+  e = by_format(f16, [&](auto fmt) {
+    constexpr bool F = decltype(fmt)::value;
+    if (R->is_sylvester) {
+      const int64_t nchunks = N * K / kVec;
+      return by_group_size(R->G, [&](auto g) {
+        constexpr int Gv = decltype(g)::value;
+        cudaError_t r = flat_launch<Gv, kFlatAbsmax, false, F>(W, nchunks, K / kVec, nullptr,
+                                                               nullptr, amax, stream);
+        if (r != cudaSuccess) return r;
+        return flat_launch<Gv, kFlatQuant, false, F>(W, nchunks, K / kVec, nullptr, Wq, amax,
+                                                     stream);
+      });
+    }
     const int64_t gpt = K / R->G;
-    e = by_group_size(R->G, [&](auto g) {
+    return by_group_size(R->G, [&](auto g) {
       constexpr int Gv = decltype(g)::value;
-      cudaError_t r = dense_launch<Gv, uint16_t, kDenseAbsmaxAll>(W, N * gpt, gpt, R->R_dev,
-                                                                  nullptr, 0, nullptr, amax, stream);
+      cudaError_t r = dense_launch<Gv, uint16_t, kDenseAbsmaxAll, F>(W, N * gpt, gpt, R->R_dev,
+                                                                     nullptr, 0, nullptr, amax,
+                                                                     stream);
       if (r != cudaSuccess) return r;
-      return dense_launch<Gv, uint16_t, kDenseQuantAll>(W, N * gpt, gpt, R->R_dev, nullptr, 0, Wq,
-                                                        amax, stream);
+      return dense_launch<Gv, uint16_t, kDenseQuantAll, F>(W, N * gpt, gpt, R->R_dev, nullptr, 0,
+                                                           Wq, amax, stream);
     });
-  }
+  });
   if (e != cudaSuccess) return e;
   finalize_scales<<<1, 32, 0, stream>>>(s_w, 1);
   return cudaGetLastError();

@@ -55,6 +55,7 @@ typedef enum convrot_status {
 } convrot_status;
 
 typedef uint16_t convrot_bf16;                     /* bfloat16 bit pattern */
+typedef uint16_t convrot_f16;                      /* IEEE binary16 (fp16) bit pattern */
 typedef void* convrot_stream_t;                    /* cudaStream_t */
 typedef struct convrot_rotation_s* convrot_rotation_t;  /* opaque, owned by the library */
 
@@ -184,6 +185,36 @@ convrot_status convrot_linear_int8_noalloc(const convrot_bf16* x, int64_t M, int
                                            convrot_stream_t stream);
 /* Size of that static scratch in bytes (CONVROT_NOALLOC_SCRATCH_BYTES). */
 size_t convrot_noalloc_scratch_bytes(void);
+
+/*
+ * fp16 forms.  The pages' int8 layers run with BF16 or FP16 activations and
+ * refuse only FP32 (Invoke docs "int8 Compute": the opening section unpacks
+ * each layer "to BF16 or FP16", and the table of layers that keep
+ * dequantizing lists "Running in FP32" alone).  Each function below is its
+ * bf16 namesake with every 16-bit float tensor in IEEE fp16 instead: the
+ * input W or x is read exactly, and the outputs W_hat and y (and the bias) are
+ * fp16, each value rounded once to nearest-even (fp16 overflow gives +-inf,
+ * tiny values fp16 subnormals).  Arguments, limits and errors are the
+ * namesake's; convrot_dequant_derotate_f16 is the correctly rounded fp16 of
+ * the exact value with the Sylvester R.
+ */
+convrot_status convrot_quantize_weight_f16(const convrot_f16* W, int64_t N, int64_t K,
+                                           convrot_rotation_t R, int8_t* Wq, float* s_w,
+                                           convrot_stream_t stream);
+convrot_status convrot_dequant_derotate_f16(const int8_t* Wq, const float* s_w, int64_t s_w_len,
+                                            int64_t N, int64_t K, convrot_rotation_t R,
+                                            convrot_f16* W_hat, convrot_stream_t stream);
+convrot_status convrot_rotate_quant_act_f16(const convrot_f16* x, int64_t M, int64_t K,
+                                            convrot_rotation_t R, int8_t* xq, float* s_tok,
+                                            convrot_stream_t stream);
+convrot_status convrot_int8_gemm_f16(const int8_t* xq, const float* s_tok, const int8_t* Wq,
+                                     const float* s_w, int64_t s_w_len, const convrot_f16* bias,
+                                     int64_t M, int64_t N, int64_t K, convrot_f16* y,
+                                     convrot_stream_t stream);
+convrot_status convrot_linear_int8_f16(const convrot_f16* x, int64_t M, int64_t K, int64_t N,
+                                       convrot_rotation_t R, const int8_t* Wq, const float* s_w,
+                                       int64_t s_w_len, const convrot_f16* bias, convrot_f16* y,
+                                       void* ws, size_t ws_bytes, convrot_stream_t stream);
 
 /* Bytes of workspace an operation needs (0 if none); 0 for an unknown op. */
 size_t convrot_workspace_bytes(int op, int64_t M, int64_t N, int64_t K);
