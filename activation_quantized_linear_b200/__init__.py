@@ -222,9 +222,10 @@ def rotate_quant_act(x: torch.Tensor, rot: Rotation, xq: torch.Tensor | None = N
 
 def int8_gemm(xq: torch.Tensor, s_tok: torch.Tensor, Wq: torch.Tensor, s_w: torch.Tensor,
               bias: torch.Tensor | None = None, out: torch.Tensor | None = None,
-              dtype: torch.dtype = torch.bfloat16) -> torch.Tensor:
-    """y = f16(xq . Wq^T * s_tok[:, None] * s_w + bias) in `dtype` (bf16 or fp16;
-    the dtype of `out` when given); bias, if any, in the same dtype."""
+              dtype: torch.dtype | None = None) -> torch.Tensor:
+    """y = xq . Wq^T * s_tok[:, None] * s_w + bias, rounded once to a 16-bit
+    float: the dtype of `out` when given, else `dtype`, else the bias's dtype,
+    else bf16.  The bias, if any, is in the output's dtype."""
     _need(xq, "xq", torch.int8, 2)
     _need(Wq, "Wq", torch.int8, 2)
     _need(s_tok, "s_tok", torch.float32, 1)
@@ -233,7 +234,9 @@ def int8_gemm(xq: torch.Tensor, s_tok: torch.Tensor, Wq: torch.Tensor, s_w: torc
     N = Wq.shape[0]
     if Wq.shape[1] != K:
         raise ValueError("xq and Wq disagree on K")
-    out = torch.empty((M, N), dtype=dtype, device=xq.device) if out is None else out
+    if out is None:
+        dtype = dtype or (bias.dtype if bias is not None else torch.bfloat16)
+        out = torch.empty((M, N), dtype=dtype, device=xq.device)
     _need16(out, "out", 2)
     if bias is not None:
         _need(bias, "bias", out.dtype, 1)

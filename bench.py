@@ -245,6 +245,7 @@ def config_dict(args, lins, gpu=True):
         "workload": args.workload,
         "linears": [f"{l.name}:M{l.M}xK{l.K}->N{l.N}" for l in lins],
         "G": lins[0].G, "rotation": "sylvester-hadamard",
+        "activations": getattr(args, "dtype", "bf16"),
     }
     if gpu:
         cfg.update({
@@ -275,7 +276,8 @@ def run_ours(args, lins):
     rot = cr.Rotation(workloads.sylvester_rotation(lins[0].G))
     layers = []
     for i, lin in enumerate(lins):
-        inp = workloads.make_layer_inputs(lin, 1 + rank)  # every rank its own tokens
+        act = torch.float16 if args.dtype == "f16" else torch.bfloat16
+        inp = workloads.make_layer_inputs(lin, 1 + rank, dtype=act)  # every rank its own tokens
         W = inp.W.to(dev)
         Wq, s_w = cr.quantize_weight(W, rot)
         del W
@@ -284,9 +286,9 @@ def run_ours(args, lins):
             bias=inp.bias.to(dev),
             xq=torch.empty((lin.M, lin.K), dtype=torch.int8, device=dev),
             s_tok=torch.empty(lin.M, dtype=torch.float32, device=dev),
-            y=torch.empty((lin.M, lin.N), dtype=torch.bfloat16, device=dev),
-            y_host=torch.empty((lin.M, lin.N), dtype=torch.bfloat16).pin_memory(),
-            W_hat=torch.empty((lin.N, lin.K), dtype=torch.bfloat16, device=dev),
+            y=torch.empty((lin.M, lin.N), dtype=act, device=dev),
+            y_host=torch.empty((lin.M, lin.N), dtype=act).pin_memory(),
+            W_hat=torch.empty((lin.N, lin.K), dtype=act, device=dev),
             ws=torch.empty(cr.workspace_bytes(lin.M, lin.N, lin.K), dtype=torch.uint8,
                            device=dev),
         ))
@@ -496,7 +498,35 @@ def run_sweep(args):
         out = torch.empty((N, K), dtype=torch.bfloat16, device="cuda")
         t = timed(lambda: cr.dequant_derotate(Wq, s_w, rot, out=out), args.steps)
         dec.append({"G": G, "ms": t, "GBps": 3 * N * K / t / 1e6, "frac_hbm": 3 * N * K / t / 1e6 / hbm_gbs})
+    # per-output-channel weight scales and fp16 activations/outputs, G = 256:
+    # the GEMM at M = 8192 and the [12288, 3072] decode
+    var = []
+    rot = cr.Rotation(workloads.sylvester_rotation(256))
+    M = 8192
+    for fmt, per_channel in (("bf16", True), ("f16", False), ("f16", True)):
+        act = torch.float16 if fmt == "f16" else torch.bfloat16
+        inp = workloads.make_layer_inputs(workloads.Linear("sweep", M, 4096, 4096), 4, dtype=act)
+        Wq, s_w = cr.quantize_weight(inp.W.cuda(), rot)
+        if per_channel:
+            s_w = (s_w * (1 + 0.1 * torch.rand(4096, device="cuda"))).contiguous()
+        x, bias = inp.x.cuda(), inp.bias.cuda()
+        xq, s_tok = cr.rotate_quant_act(x, rot)
+        y = cr.int8_gemm(xq, s_tok, Wq, s_w, bias)
+        t_r = timed(lambda: cr.rotate_quant_act(x, rot, xq=xq, s_tok=s_tok), args.steps)
+        t_g = timed(lambda: cr.int8_gemm(xq, s_tok, Wq, s_w, bias, out=y), args.steps)
+        Wd = torch.randint(-127, 128, (N, K), dtype=torch.int8, device="cuda")
+        sd = (torch.rand(N, device="cuda") * 1e-3 + 1e-4) if per_channel else torch.tensor([1e-3], device="cuda")
+        out = torch.empty((N, K), dtype=act, device="cuda")
+        t_d = timed(lambda: cr.dequant_derotate(Wd, sd, rot, out=out), args.steps)
+        ops = 2.0 * M * 4096 * 4096
+        var.append({"activations": fmt, "s_w": "per_channel" if per_channel else "per_tensor",
+                    "rotate_ms": t_r, "rotate_GBps": (3 * M * 4096 + 4 * M) / t_r / 1e6,
+                    "gemm_ms": t_g, "gemm_TOPS": ops / t_g / 1e9,
+                    "gemm_frac_int8_peak": ops / t_g / 1e9 / int8_peak,
+                    "decode_12288x3072_ms": t_d, "decode_GBps": 3 * N * K / t_d / 1e6,
+                    "decode_frac_hbm": 3 * N * K / t_d / 1e6 / hbm_gbs})
     print(json.dumps({"sweep": "group_size_and_skinny_M", "linears": rows, "decode_12288x3072": dec,
+                      "variants_G256": var,
                       "peaks": {"hbm_gbs": hbm_gbs, "int8_tops": int8_peak}}))
     return 0
 
@@ -509,6 +539,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="zimage_dit_block",
                     choices=[k for k in workloads.WORKLOADS if k != "group_size_sweep"])
+    ap.add_argument("--dtype", default="bf16", choices=["bf16", "f16"],
+                    help="16-bit float format of activations, bias, outputs and the decoded weight")
     ap.add_argument("--ref-rows", type=int, default=64)
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
