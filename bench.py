@@ -525,8 +525,24 @@ def run_sweep(args):
                     "gemm_frac_int8_peak": ops / t_g / 1e9 / int8_peak,
                     "decode_12288x3072_ms": t_d, "decode_GBps": 3 * N * K / t_d / 1e6,
                     "decode_frac_hbm": 3 * N * K / t_d / 1e6 / hbm_gbs})
+    # a dense (non-Hadamard) orthogonal R: the float64 FMA path
+    dense = []
+    for G in (64, 256):
+        rot = cr.Rotation(workloads.qr_rotation(G))
+        inp = workloads.make_layer_inputs(workloads.Linear("sweep", M, 4096, 4096, G=G), 4)
+        x = inp.x.cuda()
+        xq, s_tok = cr.rotate_quant_act(x, rot)
+        t_r = timed(lambda: cr.rotate_quant_act(x, rot, xq=xq, s_tok=s_tok), max(3, args.steps // 4))
+        Wd = torch.randint(-127, 128, (N, K), dtype=torch.int8, device="cuda")
+        sd = torch.tensor([1e-3], device="cuda")
+        out = torch.empty((N, K), dtype=torch.bfloat16, device="cuda")
+        t_d = timed(lambda: cr.dequant_derotate(Wd, sd, rot, out=out), max(3, args.steps // 4))
+        dense.append({"G": G, "rotate_ms": t_r, "rotate_GBps": (3 * M * 4096 + 4 * M) / t_r / 1e6,
+                      "rotate_fp64_tflops": 2.0 * G * M * 4096 * 2 / t_r / 1e9,
+                      "decode_12288x3072_ms": t_d, "decode_GBps": 3 * N * K / t_d / 1e6,
+                      "decode_fp64_tflops": 2.0 * G * N * K / t_d / 1e9})
     print(json.dumps({"sweep": "group_size_and_skinny_M", "linears": rows, "decode_12288x3072": dec,
-                      "variants_G256": var,
+                      "variants_G256": var, "dense_R_M8192": dense,
                       "peaks": {"hbm_gbs": hbm_gbs, "int8_tops": int8_peak}}))
     return 0
 

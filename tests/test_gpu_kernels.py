@@ -325,3 +325,38 @@ def test_layer_module_two_modes_agree():
 
 def test_check_status_clean():
     cr.check_status()
+
+
+# ---------------------------------------------------------------------------
+# CUDA graphs: the int8-compute forward captured once and replayed
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("M", [64, 300])
+def test_linear_int8_cuda_graph_replay(M):
+    """convrot_linear_int8 (rotate+quantize, chained GEMM) captured in a CUDA
+    graph and replayed on new inputs written into the captured buffers gives the
+    eager results bit for bit."""
+    lin = workloads.Linear("graph", M, 1024, 2048, G=256)
+    inp = workloads.make_layer_inputs(lin, 3)
+    rot = cr.Rotation(inp.R)
+    Wq, s_w = cr.quantize_weight(inp.W.cuda(), rot)
+    bias = inp.bias.cuda()
+    x = inp.x.cuda()
+    ws = torch.empty(cr.workspace_bytes(M, lin.N, lin.K), dtype=torch.uint8, device="cuda")
+    y = torch.empty((M, lin.N), dtype=torch.bfloat16, device="cuda")
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):  # warm-up off the capture stream, as torch asks
+        cr.linear_int8(x, Wq, s_w, rot, bias, out=y, workspace=ws)
+    torch.cuda.current_stream().wait_stream(side)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        cr.linear_int8(x, Wq, s_w, rot, bias, out=y, workspace=ws)
+    for seed in (11, 12):
+        x_new = workloads.make_activation(M, lin.K, seed=seed).cuda()
+        x.copy_(x_new)
+        graph.replay()
+        torch.cuda.synchronize()
+        y_eager = cr.linear_int8(x_new, Wq, s_w, rot, bias)
+        torch.cuda.synchronize()
+        assert torch.equal(y.view(torch.int16), y_eager.view(torch.int16))
+    cr.check_status()
