@@ -53,7 +53,7 @@ def _load() -> ctypes.CDLL:
     path = _build.LIB_PATH
     if not os.path.exists(path):
         raise ImportError(
-            f"{path} is missing: build it with `python -m activation_quantized_linear_b200.build`"
+            f"{path} is missing: build it with `python activation_quantized_linear_b200/build.py`"
             " (the layer has no CPU fallback)")
     lib = ctypes.CDLL(path)
     vp, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
@@ -74,6 +74,7 @@ def _load() -> ctypes.CDLL:
         "convrot_linear_int8_noalloc": ([vp, i64, i64, i64, vp, vp, vp, i64, vp, vp, vp], i32),
         "convrot_noalloc_scratch_bytes": ([], sz),
         "convrot_check_status": ([vp], i32),
+        "convrot_selftest_wait_timeout": ([i32, vp], i32),
         "convrot_quantize_weight_f16": ([vp, i64, i64, vp, vp, vp, vp], i32),
         "convrot_dequant_derotate_f16": ([vp, vp, i64, i64, i64, vp, vp, vp], i32),
         "convrot_rotate_quant_act_f16": ([vp, i64, i64, vp, vp, vp, vp], i32),
@@ -313,6 +314,12 @@ def check_status(stream: torch.cuda.Stream | None = None) -> None:
     """Synchronize and raise if a kernel gave up a bounded wait since the last check."""
     s = (stream or torch.cuda.current_stream()).cuda_stream
     _check(_lib.convrot_check_status(s))
+
+
+def selftest_wait_timeout(limit_ms: int = 20) -> None:
+    """Enqueue the failure-detection self-test: a kernel whose bounded wait runs
+    out after `limit_ms`; the next check_status() raises ConvRotError(TIMEOUT)."""
+    _check(_lib.convrot_selftest_wait_timeout(int(limit_ms), _stream()))
 
 
 class ConvRotLinear:

@@ -1,6 +1,7 @@
 """Build libconvrot.so in place with nvcc for sm_100a.
 
-Usage: python -m activation_quantized_linear_b200.build [--verbose] [--ptxas-info]
+Usage: python activation_quantized_linear_b200/build.py [--verbose] [--ptxas-info]
+(run as a script: importing the package loads the library it builds)
 
 The library links the CUDA runtime statically and reaches the driver API only
 through cudaGetDriverEntryPoint, so it loads on a machine without a GPU (the

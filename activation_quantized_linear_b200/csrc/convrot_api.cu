@@ -438,6 +438,18 @@ convrot_status convrot_linear_int8_f16(const convrot_f16* x, int64_t M, int64_t 
   return linear_int8_impl(x, true, M, K, N, R, Wq, s_w, s_w_len, bias, y, ws, ws_bytes, stream);
 }
 
+convrot_status convrot_selftest_wait_timeout(int limit_ms, convrot_stream_t stream) {
+  if (limit_ms < 1 || limit_ms > 1000) {
+    return fail(CONVROT_ERR_INVALID_ARG, "limit_ms=%d must be in [1, 1000]", limit_ms);
+  }
+  int dev = -1;
+  convrot_status s = current_device(&dev);
+  if (s != CONVROT_OK) return s;
+  return launched(convrot::launch_bounded_wait_selftest(
+                      static_cast<uint64_t>(limit_ms) * 1000000ull, as_stream(stream)),
+                  "selftest_wait_timeout launch");
+}
+
 convrot_status convrot_check_status(convrot_stream_t stream) {
   unsigned int st = 0;
   cudaError_t e = convrot::read_and_clear_status(&st, as_stream(stream));

@@ -60,6 +60,10 @@ cudaError_t launch_int8_gemm(const GemmArgs& a, cudaStream_t stream);
 // The few-token variant (M <= 128): swap-AB with the K split over a cluster.
 cudaError_t launch_int8_gemm_skinny(const GemmArgs& a, cudaStream_t stream);
 
+// Enqueues the failure-detection self-test: a bounded wait that runs out
+// after `limit_ns` and records a timeout in the status word.
+cudaError_t launch_bounded_wait_selftest(uint64_t limit_ns, cudaStream_t stream);
+
 // Reads and clears the current device's kernel status word (0 = fine).
 cudaError_t read_and_clear_status(unsigned int* status, cudaStream_t stream);
 

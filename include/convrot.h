@@ -226,6 +226,18 @@ size_t convrot_workspace_bytes(int op, int64_t M, int64_t N, int64_t K);
  */
 convrot_status convrot_check_status(convrot_stream_t stream);
 
+/*
+ * Failure-detection self-test (no counterpart on the pages: it tests this
+ * library's own timeout reporting).  Enqueues one small kernel whose bounded
+ * wait can never be satisfied: it gives up after `limit_ms` milliseconds
+ * (1..1000, else CONVROT_ERR_INVALID_ARG) and records a timeout in the
+ * device status word, as a kernel whose pipeline stalled would.  Returns
+ * CONVROT_OK once enqueued; the next convrot_check_status on the stream then
+ * reports CONVROT_ERR_TIMEOUT and clears the word.  Nothing faults or hangs,
+ * and the context stays usable.
+ */
+convrot_status convrot_selftest_wait_timeout(int limit_ms, convrot_stream_t stream);
+
 /* Message of the last failure on the calling thread ("" if none). */
 const char* convrot_last_error_string(void);
 

@@ -360,3 +360,24 @@ def test_linear_int8_cuda_graph_replay(M):
         torch.cuda.synchronize()
         assert torch.equal(y.view(torch.int16), y_eager.view(torch.int16))
     cr.check_status()
+
+
+# ---------------------------------------------------------------------------
+# failure detection: a bounded wait that runs out is reported, nothing hangs
+# ---------------------------------------------------------------------------
+def test_bounded_wait_timeout_is_reported():
+    cr.check_status()  # clean to start with
+    cr.selftest_wait_timeout(20)
+    with pytest.raises(cr.ConvRotError) as e:
+        cr.check_status()
+    assert e.value.status == cr.TIMEOUT
+    cr.check_status()  # reading the status cleared it
+    with pytest.raises(cr.ConvRotError) as e:
+        cr.selftest_wait_timeout(0)
+    assert e.value.status == cr.INVALID_ARG
+    # the context still computes: a small GEMM, bit-exact
+    rng = np.random.default_rng(99)
+    a, b = _codes(rng, (65, 256)), _codes(rng, (144, 256))
+    acc = cr.int8_gemm_s32(torch.from_numpy(a).cuda(), torch.from_numpy(b).cuda())
+    np.testing.assert_array_equal(acc.cpu().numpy(), oracle.int8_gemm_acc(a, b))
+    cr.check_status()
