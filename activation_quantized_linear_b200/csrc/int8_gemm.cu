@@ -5,7 +5,7 @@
 //   acc[m, n] = sum_k xq[m, k] * Wq[n, k]                       (exact int32)
 //   y[m, n]   = bf16_rn(float(acc) * (s_tok[m] * s_w[n|0]) + bias[n])
 //
-// Structure (persistent; one CTA per SM):
+// Structure (persistent; one CTA per SM, CTA pairs as clusters of two SMs):
 //   warp 0      TMA producer: A and B int8 tiles of 128-byte rows, 128-byte
 //               swizzle, into a shared-memory ring;
 //   warp 1      allocates 512 TMEM columns; one thread issues tcgen05.mma
@@ -15,11 +15,12 @@
 //   warps 2..5  epilogue: tcgen05.ld 32 columns at a time, rescale, bias, bf16,
 //               128-bit global stores; then release the accumulator so the MMA
 //               of the next tile overlaps this tile's epilogue.
-// For more than 128 tokens, CTA pairs (clusters of two SMs, cta_group::2) work
-// on 256 x 256 tiles: each CTA loads its 128 rows of A and 128 rows of B (no
-// multicast), the even CTA issues M=256 x N=256 MMAs whose accumulators are
-// split across the two CTAs' TMEM, and commits signal both CTAs' barriers.  A
-// pair moves 2/3 of the operand bytes per MMA that two single CTAs would.
+// A CTA pair (cta_group::2) works on 256 x 256 tiles: each CTA loads its 128
+// rows of A and 128 rows of B (no multicast), the even CTA issues M=256 x
+// N=256 MMAs whose accumulators are split across the two CTAs' TMEM, and
+// commits signal both CTAs' barriers.  A pair moves 2/3 of the operand bytes
+// per MMA that two single CTAs would.  (Up to 128 tokens take the swap-AB
+// kernel in int8_gemm_skinny.cu instead.)
 // Every mbarrier wait is bounded by the global timer.  A wait that runs out
 // records CONVROT_ERR_TIMEOUT in the device status word; the CTA then stops
 // issuing work, drains what it issued and frees its TMEM before returning.
@@ -48,22 +49,19 @@ constexpr int kThreads = 192;
 constexpr int kEpiWarps = 4;
 constexpr uint64_t kWaitNs = 1000000000ull;  // 1 s per wait
 
-// Two variants share the kernel body:
-//   single: one CTA per tile of 128 x 256, B tile 256 x 128 per stage, 4 stages;
-//   pair:   a cluster of two CTAs per tile of 256 x 256 (cta_group::2); each CTA
-//           loads its 128 rows of A and its 128 rows of B per stage, 6 stages,
-//           and only the even CTA issues the MMAs.
-template <bool PAIR>
+// A cluster of two CTAs per tile of 256 x 256 (cta_group::2); each CTA loads
+// its 128 rows of A and its 128 rows of B per stage, 6 stages, and only the
+// even CTA issues the MMAs.
 struct Cfg {
-  static constexpr int kBRows = PAIR ? BN / 2 : BN;   // B rows loaded per CTA
+  static constexpr int kBRows = BN / 2;  // B rows loaded per CTA
   static constexpr int kBStage = kBRows * BK;
   static constexpr int kStageBytes = A_STAGE + kBStage;
-  static constexpr int kStages = PAIR ? 6 : 4;
-  static constexpr int kTileM = PAIR ? 2 * BM : BM;
+  static constexpr int kStages = 6;
+  static constexpr int kTileM = 2 * BM;
   static constexpr size_t kSmem = 1024 + kStages * kStageBytes + 256;
   static constexpr uint32_t kIdesc = ptx::idesc_i8(kTileM, BN);
-  // bytes that complete one stage on the (leader's) full barrier
-  static constexpr uint32_t kTxBytes = (PAIR ? 2 : 1) * kStageBytes;
+  // bytes that complete one stage on the leader's full barrier (both CTAs' loads)
+  static constexpr uint32_t kTxBytes = 2 * kStageBytes;
 };
 
 struct Params {
@@ -163,11 +161,10 @@ __device__ __forceinline__ void store_s32_row32(int32_t* dst, const uint32_t (&r
   }
 }
 
-template <bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
     int8_gemm_tcgen05(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                       const Params p) {
-  using C = Cfg<PAIR>;
+  using C = Cfg;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -178,10 +175,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const uint32_t lane = threadIdx.x & 31;
-  const uint32_t rank = PAIR ? ptx::cluster_ctarank() : 0;  // CTA within the pair
+  const uint32_t rank = ptx::cluster_ctarank();  // CTA within the pair
   const bool leader = rank == 0;
-  const int unit = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
-  const int units = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
+  const int unit = static_cast<int>(blockIdx.x >> 1);
+  const int units = static_cast<int>(gridDim.x >> 1);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
@@ -190,7 +187,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       ptx::mbar_init(&bars->acc_full[a], 1);
-      ptx::mbar_init(&bars->acc_empty[a], (PAIR ? 2 : 1) * kEpiWarps);
+      ptx::mbar_init(&bars->acc_empty[a], 2 * kEpiWarps);
     }
     ptx::mbar_init(&bars->drain, 1);
     bars->abort_flag = 0;
@@ -199,20 +196,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::tma_prefetch_desc(&tmB);
   }
   if (warp == 1) {
-    if constexpr (PAIR) {
-      ptx::tmem_alloc_pair(&bars->tmem_base, TMEM_COLS);
-      ptx::tmem_relinquish_pair();
-    } else {
-      ptx::tmem_alloc(&bars->tmem_base, TMEM_COLS);
-      ptx::tmem_relinquish();
-    }
+    ptx::tmem_alloc_pair(&bars->tmem_base, TMEM_COLS);
+    ptx::tmem_relinquish_pair();
   }
   ptx::tc_fence_before();
-  if constexpr (PAIR) {
-    ptx::cluster_sync();  // both CTAs' barriers initialised before any cross-CTA signal
-  } else {
-    __syncthreads();
-  }
+  ptx::cluster_sync();  // both CTAs' barriers initialised before any cross-CTA signal
   ptx::tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
   const int num_tiles = p.m_tiles * p.n_tiles;
@@ -238,15 +226,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           record_timeout(abort_flag, p.status);
           break;
         }
-        if constexpr (PAIR) {
-          if (leader) ptx::mbar_arrive_expect_tx(&bars->full[stage], C::kTxBytes);
-          ptx::tma_load_2d_pair(sA + stage * A_STAGE, &tmA, &bars->full[stage], kb * BK, a_row);
-          ptx::tma_load_2d_pair(sB + stage * C::kBStage, &tmB, &bars->full[stage], kb * BK, b_row);
-        } else {
-          ptx::mbar_arrive_expect_tx(&bars->full[stage], C::kTxBytes);
-          ptx::tma_load_2d(sA + stage * A_STAGE, &tmA, &bars->full[stage], kb * BK, a_row);
-          ptx::tma_load_2d(sB + stage * C::kBStage, &tmB, &bars->full[stage], kb * BK, b_row);
-        }
+        if (leader) ptx::mbar_arrive_expect_tx(&bars->full[stage], C::kTxBytes);
+        ptx::tma_load_2d_pair(sA + stage * A_STAGE, &tmA, &bars->full[stage], kb * BK, a_row);
+        ptx::tma_load_2d_pair(sB + stage * C::kBStage, &tmB, &bars->full[stage], kb * BK, b_row);
         last_stage = stage;
         last_phase = phase;
         if (++stage == C::kStages) {
@@ -288,37 +270,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int k = 0; k < BK / UMMA_K; ++k) {
           const uint64_t ad = ptx::smem_desc_k_sw128(a_addr + k * UMMA_K);
           const uint64_t bd = ptx::smem_desc_k_sw128(b_addr + k * UMMA_K);
-          if constexpr (PAIR) {
-            ptx::mma_i8_pair(d_tmem, ad, bd, C::kIdesc, (kb | k) != 0 ? 1u : 0u);
-          } else {
-            ptx::mma_i8(d_tmem, ad, bd, C::kIdesc, (kb | k) != 0 ? 1u : 0u);
-          }
+          ptx::mma_i8_pair(d_tmem, ad, bd, C::kIdesc, (kb | k) != 0 ? 1u : 0u);
         }
         issued = true;
-        if constexpr (PAIR) {
-          ptx::mma_commit_pair(&bars->empty[stage]);
-        } else {
-          ptx::mma_commit(&bars->empty[stage]);
-        }
+        ptx::mma_commit_pair(&bars->empty[stage]);
         if (++stage == C::kStages) {
           stage = 0;
           phase ^= 1u;
         }
       }
       if (!ok) break;
-      if constexpr (PAIR) {
-        ptx::mma_commit_pair(&bars->acc_full[acc]);
-      } else {
-        ptx::mma_commit(&bars->acc_full[acc]);
-      }
+      ptx::mma_commit_pair(&bars->acc_full[acc]);
     }
     if (*abort_flag && issued) {
       // every MMA issued so far must finish before TMEM is released
-      if constexpr (PAIR) {
-        ptx::mma_commit_pair_local(&bars->drain);
-      } else {
-        ptx::mma_commit(&bars->drain);
-      }
+      ptx::mma_commit_pair_local(&bars->drain);
       ptx::mbar_wait(&bars->drain, 0, ptx::globaltimer_ns() + 10000000ull);
     }
   } else if (warp >= 2) {
@@ -361,30 +327,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       ptx::tc_fence_before();
       __syncwarp();
-      if (lane == 0) {
-        if constexpr (PAIR) {
-          ptx::mbar_arrive_leader(&bars->acc_empty[acc]);
-        } else {
-          ptx::mbar_arrive(&bars->acc_empty[acc]);
-        }
-      }
+      if (lane == 0) ptx::mbar_arrive_leader(&bars->acc_empty[acc]);
     }
   }
 
   ptx::tc_fence_before();
-  if constexpr (PAIR) {
-    ptx::cluster_sync();  // the leader's MMAs into this CTA's TMEM are complete
-  } else {
-    __syncthreads();
-  }
+  ptx::cluster_sync();  // the leader's MMAs into this CTA's TMEM are complete
   if (warp == 1) {
     __syncwarp();
     ptx::tc_fence_after();
-    if constexpr (PAIR) {
-      ptx::tmem_dealloc_pair(tmem, TMEM_COLS);
-    } else {
-      ptx::tmem_dealloc(tmem, TMEM_COLS);
-    }
+    ptx::tmem_dealloc_pair(tmem, TMEM_COLS);
   }
 }
 
@@ -396,15 +348,14 @@ bool encode_operand(CUtensorMap* map, const int8_t* base, int64_t rows, int64_t 
                        static_cast<uint32_t>(box_rows));
 }
 
-template <bool PAIR>
-cudaError_t launch_variant(const GemmArgs& a, Params p, cudaStream_t stream) {
-  using C = Cfg<PAIR>;
+cudaError_t launch_pair(const GemmArgs& a, Params p, cudaStream_t stream) {
+  using C = Cfg;
   CUtensorMap tmA, tmB;
   if (!encode_operand(&tmA, a.A, a.M, a.K, BM) ||
       !encode_operand(&tmB, a.B, a.N, a.K, C::kBRows)) {
     return cudaErrorInvalidValue;
   }
-  cudaError_t e = cudaFuncSetAttribute(int8_gemm_tcgen05<PAIR>,
+  cudaError_t e = cudaFuncSetAttribute(int8_gemm_tcgen05,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(C::kSmem));
   if (e != cudaSuccess) return e;
@@ -412,7 +363,7 @@ cudaError_t launch_variant(const GemmArgs& a, Params p, cudaStream_t stream) {
   // all M-tiles per column sweep when A (M x K bytes) fits in half of L2
   p.group_m = a.M * a.K <= (64ll << 20) ? p.m_tiles : 8;
   const int tiles = p.m_tiles * p.n_tiles;
-  const int per_unit = PAIR ? 2 : 1;
+  const int per_unit = 2;  // CTAs per cluster
   const int max_units = sm_count() / per_unit;
   const int units = tiles < max_units ? tiles : max_units;
   cudaLaunchConfig_t cfg = {};
@@ -429,7 +380,7 @@ cudaError_t launch_variant(const GemmArgs& a, Params p, cudaStream_t stream) {
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, int8_gemm_tcgen05<PAIR>, tmA, tmB, p);
+  return cudaLaunchKernelEx(&cfg, int8_gemm_tcgen05, tmA, tmB, p);
 }
 
 }  // namespace
@@ -453,7 +404,7 @@ cudaError_t launch_int8_gemm(const GemmArgs& a, cudaStream_t stream) {
   // few tokens: the weight-streaming swap-AB kernel; otherwise CTA pairs
   // (256-row tiles) once there is more than one 128-row block of tokens
   if (a.M <= BM) return launch_int8_gemm_skinny(a, stream);
-  return launch_variant<true>(a, p, stream);
+  return launch_pair(a, p, stream);
 }
 
 }  // namespace convrot
