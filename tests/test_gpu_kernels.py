@@ -72,13 +72,15 @@ def test_int8_gemm_s32_bit_exact(M, N, K):
     np.testing.assert_array_equal(acc.cpu().numpy(), oracle.int8_gemm_acc(a, b))
 
 
-def test_int8_gemm_s32_extremes():
-    """Largest accumulators of the workloads (|acc| = 127^2 K, K = 15360)."""
-    K = 15360
-    a = np.full((130, K), 127, np.int8)
+@pytest.mark.parametrize("M,N,K", [(130, 272, 15360), (130, 144, 131072), (3, 144, 131072)])
+def test_int8_gemm_s32_extremes(M, N, K):
+    """Largest accumulators: |acc| = 127^2 K, at the workloads' K = 15360 and at
+    the interface's limit K = 131072 (127^2 * 131072 < 2^31), on both GEMM
+    paths (CTA pairs for M > 128, swap-AB below)."""
+    a = np.full((M, K), 127, np.int8)
     a[1::2] = -127
-    a[5, ::2] = 0
-    b = np.full((272, K), 127, np.int8)
+    a[min(5, M - 1), ::2] = 0
+    b = np.full((N, K), 127, np.int8)
     b[3] = -127
     b[7, :100] = 0
     acc = cr.int8_gemm_s32(torch.from_numpy(a).cuda(), torch.from_numpy(b).cuda())
@@ -152,7 +154,8 @@ RQA_CASES = [
     for G in (4, 16, 64, 256) for kind in ("sylvester", "qr")
     for (M, K) in ((1, 256), (7, 1024), (129, 3840))
 ] + [(256, "sylvester", 33, 15360), (256, "sylvester", 17, 32768), (64, "sylvester", 20, 12288),
-     (256, "qr", 9, 10240), (16, "sylvester", 65, 5120), (256, "sylvester", 300, 2048)]
+     (256, "qr", 9, 10240), (16, "sylvester", 65, 5120), (256, "sylvester", 300, 2048),
+     (256, "sylvester", 3001, 3840)]  # several persistent row-block passes, half-empty last block
 
 
 @pytest.mark.parametrize("G,kind,M,K", RQA_CASES)
@@ -211,7 +214,8 @@ def test_quantize_weight_parity(G, kind, N, K):
     assert_codes_close(Wq.cpu().numpy(), ref_q)
 
 
-@pytest.mark.parametrize("G,kind,N,K", WQ_CASES + [(256, "sylvester", 12288 // 8, 3072)])
+@pytest.mark.parametrize("G,kind,N,K", WQ_CASES + [(256, "sylvester", 12288 // 8, 3072),
+                                                   (64, "sylvester", 4999, 3840)])
 def test_dequant_derotate_parity(G, kind, N, K):
     R = _rotation(G, kind)
     rot = cr.Rotation(R)
