@@ -5,15 +5,18 @@ provides device memory and the current stream only; every step of the layer
 runs in the library's CUDA kernels.  There is no CPU fallback: if the library
 is missing, importing the binding raises.
 
-Entry points (same names as the C ABI, without the `convrot_` prefix):
+Entry points (same names as the C ABI, without the `convrot_` prefix; the
+16-bit float tensors may be bf16 or fp16, which selects the `_f16` C entry):
     Rotation(R)                               the G x G rotation block, on the current device
     quantize_weight(W, rot)          -> (Wq, s_w)
-    dequant_derotate(Wq, s_w, rot)   -> W_hat (bf16)
+    dequant_derotate(Wq, s_w, rot)   -> W_hat (bf16, or `dtype` / out's dtype)
     rotate_quant_act(x, rot)         -> (xq, s_tok)
-    int8_gemm(xq, s_tok, Wq, s_w, bias)      -> y (bf16)
+    int8_gemm(xq, s_tok, Wq, s_w, bias)      -> y (out's, `dtype`'s or bias's dtype; bf16 by default)
     int8_gemm_s32(xq, Wq)                    -> acc (int32)
-    linear_int8(x, Wq, s_w, rot, bias)       -> y (bf16)
-    workspace_bytes(M, N, K), check_status()
+    linear_int8(x, Wq, s_w, rot, bias)       -> y (x's dtype)
+    linear_int8_noalloc(x, Wq, s_w, rot, bias) -> y (bf16; the library's static scratch)
+    workspace_bytes(M, N, K), check_status(), selftest_wait_timeout(ms)
+    ConvRotLinear(W, R, bias)                 the layer: forward (int8 compute), decode_weight
 """
 
 from __future__ import annotations
@@ -30,7 +33,7 @@ __all__ = [
     "ConvRotError", "Rotation", "quantize_weight", "dequant_derotate", "rotate_quant_act",
     "int8_gemm", "int8_gemm_s32", "linear_int8", "workspace_bytes", "check_status",
     "device_supported", "library_path", "ConvRotLinear", "linear_int8_noalloc",
-    "noalloc_scratch_bytes",
+    "noalloc_scratch_bytes", "selftest_wait_timeout",
 ]
 
 OK, INVALID_ARG, UNSUPPORTED, CUDA, WORKSPACE, TIMEOUT, ALIGNMENT = range(7)

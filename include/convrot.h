@@ -130,7 +130,7 @@ convrot_status convrot_rotate_quant_act(const convrot_bf16* x, int64_t M, int64_
  *   y[m, n]   = bf16_rn( float(acc) * (s_tok[m] * s_w[n or 0]) + bias[n] )
  * xq [M, K] int8, s_tok [M] f32, Wq [N, K] int8, s_w f32 (s_w_len = 1 or N),
  * bias [N] bf16 or NULL; y [M, N] bf16 out.  K % 16 == 0, K <= 131072,
- * N % 16 == 0, M >= 0.  No workspace is needed (ws may be NULL / 0).
+ * N % 16 == 0, M >= 0.  No workspace is needed.
  */
 convrot_status convrot_int8_gemm(const int8_t* xq, const float* s_tok, const int8_t* Wq,
                                  const float* s_w, int64_t s_w_len, const convrot_bf16* bias,
