@@ -37,7 +37,7 @@ __all__ = [
 ]
 
 OK, INVALID_ARG, UNSUPPORTED, CUDA, WORKSPACE, TIMEOUT, ALIGNMENT = range(7)
-OP_LINEAR_INT8 = 1
+OP_LINEAR_INT8, OP_LINEAR_INT8_SLICED = 1, 2
 STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "CUDA", 4: "WORKSPACE",
                 5: "TIMEOUT", 6: "ALIGNMENT"}
 
@@ -263,8 +263,11 @@ def int8_gemm_s32(xq: torch.Tensor, Wq: torch.Tensor, out: torch.Tensor | None =
     return out
 
 
-def workspace_bytes(M: int, N: int, K: int) -> int:
-    return int(_lib.convrot_workspace_bytes(OP_LINEAR_INT8, M, N, K))
+def workspace_bytes(M: int, N: int, K: int, sliced: bool = False) -> int:
+    """Workspace of linear_int8 for all M tokens at once, or (sliced=True) for
+    slices of at most 2N tokens; any size down to one row works."""
+    op = OP_LINEAR_INT8_SLICED if sliced else OP_LINEAR_INT8
+    return int(_lib.convrot_workspace_bytes(op, M, N, K))
 
 
 def linear_int8(x: torch.Tensor, Wq: torch.Tensor, s_w: torch.Tensor, rot: Rotation,

@@ -387,11 +387,21 @@ convrot_status convrot_int8_gemm_s32(const int8_t* xq, const int8_t* Wq, int64_t
   return gemm_common(xq, nullptr, Wq, nullptr, 1, nullptr, M, N, K, acc, true, false, stream);
 }
 
+// Workspace of a slice of `rows` tokens: the int8 codes, then (256-byte
+// aligned) the per-token scales.
+static size_t slice_bytes(int64_t rows, int64_t K) {
+  return align256(static_cast<size_t>(rows) * static_cast<size_t>(K)) +
+         align256(sizeof(float) * static_cast<size_t>(rows));
+}
+
 size_t convrot_workspace_bytes(int op, int64_t M, int64_t N, int64_t K) {
-  (void)N;
-  if (op != CONVROT_OP_LINEAR_INT8 || M < 0 || K < 0) return 0;
-  return align256(static_cast<size_t>(M) * static_cast<size_t>(K)) +
-         align256(sizeof(float) * static_cast<size_t>(M));
+  if (M < 0 || K < 0 || N < 0) return 0;
+  if (op == CONVROT_OP_LINEAR_INT8) return slice_bytes(M, K);
+  if (op == CONVROT_OP_LINEAR_INT8_SLICED) {
+    const int64_t rows = M < 2 * N ? M : 2 * N;
+    return slice_bytes(rows, K);
+  }
+  return 0;
 }
 
 static convrot_status linear_int8_impl(const uint16_t* x, bool f16, int64_t M, int64_t K,
@@ -409,19 +419,28 @@ static convrot_status linear_int8_impl(const uint16_t* x, bool f16, int64_t M, i
                 (long long)convrot::kMaxRotateK);
   }
   if (M == 0) return CONVROT_OK;
-  const size_t need = convrot_workspace_bytes(CONVROT_OP_LINEAR_INT8, M, N, K);
-  if (ws == nullptr || ws_bytes < need) {
-    return fail(CONVROT_ERR_WORKSPACE, "workspace of %zu bytes given, %zu needed", ws_bytes, need);
+  if (ws == nullptr || ws_bytes < slice_bytes(1, K)) {
+    return fail(CONVROT_ERR_WORKSPACE, "workspace of %zu bytes given, at least %zu needed",
+                ws_bytes, slice_bytes(1, K));
   }
   if (reinterpret_cast<uintptr_t>(ws) & 255u) {
     return fail(CONVROT_ERR_WORKSPACE, "workspace is not 256-byte aligned");
   }
+  // as many tokens per slice as the workspace holds (all of M when it fits)
+  int64_t rows = static_cast<int64_t>(ws_bytes / (static_cast<size_t>(K) + sizeof(float)));
+  if (rows > M) rows = M;
+  while (rows > 1 && slice_bytes(rows, K) > ws_bytes) --rows;
   int8_t* xq = static_cast<int8_t*>(ws);
   float* s_tok = reinterpret_cast<float*>(static_cast<char*>(ws) +
-                                          align256(static_cast<size_t>(M) * static_cast<size_t>(K)));
-  s = rotate_quant_act_impl(x, f16, M, K, R, xq, s_tok, stream);
-  if (s != CONVROT_OK) return s;
-  return gemm_common(xq, s_tok, Wq, s_w, s_w_len, bias, M, N, K, y, false, f16, stream);
+                                          align256(static_cast<size_t>(rows) * static_cast<size_t>(K)));
+  for (int64_t m0 = 0; m0 < M; m0 += rows) {
+    const int64_t r = M - m0 < rows ? M - m0 : rows;
+    s = rotate_quant_act_impl(x + m0 * K, f16, r, K, R, xq, s_tok, stream);
+    if (s != CONVROT_OK) return s;
+    s = gemm_common(xq, s_tok, Wq, s_w, s_w_len, bias, r, N, K, y + m0 * N, false, f16, stream);
+    if (s != CONVROT_OK) return s;
+  }
+  return CONVROT_OK;
 }
 
 convrot_status convrot_linear_int8(const convrot_bf16* x, int64_t M, int64_t K, int64_t N,

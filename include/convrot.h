@@ -60,7 +60,8 @@ typedef void* convrot_stream_t;                    /* cudaStream_t */
 typedef struct convrot_rotation_s* convrot_rotation_t;  /* opaque, owned by the library */
 
 /* Workspace queries (convrot_workspace_bytes). */
-#define CONVROT_OP_LINEAR_INT8 1
+#define CONVROT_OP_LINEAR_INT8 1         /* all M tokens in one pass */
+#define CONVROT_OP_LINEAR_INT8_SLICED 2  /* slices of at most 2N tokens (see convrot_linear_int8) */
 
 /* Library version, major * 10000 + minor * 100 + patch. */
 int convrot_version(void);
@@ -148,8 +149,16 @@ convrot_status convrot_int8_gemm_s32(const int8_t* xq, const int8_t* Wq, int64_t
  * The whole int8-compute forward (Invoke docs "int8 Compute"): rotate+quantize
  * x into the workspace, then the int8 GEMM with the fused epilogue.
  * x [M, K] bf16, Wq [N, K] int8, s_w (1 or N), bias [N] or NULL -> y [M, N] bf16.
- * `ws` must hold convrot_workspace_bytes(CONVROT_OP_LINEAR_INT8, M, N, K) bytes
- * (the int8 codes and the per-token scales), 256-byte aligned, else
+ * `ws` (256-byte aligned) holds the int8 codes and per-token scales of a slice
+ * of tokens: convrot_workspace_bytes(CONVROT_OP_LINEAR_INT8, M, N, K) bytes
+ * take all M tokens in one pass; a smaller workspace makes the call process
+ * the tokens in consecutive slices of as many rows as fit (the result is the
+ * same bit for bit: every row is quantized and multiplied independently).
+ * convrot_workspace_bytes(CONVROT_OP_LINEAR_INT8_SLICED, M, N, K) sizes slices
+ * of at most 2N tokens, so that the codes never take more memory than the
+ * N x K bf16 weight the default path decodes (Invoke docs "int8 Compute",
+ * "Memory": the input is quantized in slices of at most twice the layer's
+ * output width).  Less than one row's worth, or a misaligned workspace, is
  * CONVROT_ERR_WORKSPACE.  The same limits as the two steps apply.
  */
 convrot_status convrot_linear_int8(const convrot_bf16* x, int64_t M, int64_t K, int64_t N,

@@ -99,6 +99,10 @@ def test_workspace_size():
     assert need >= M * K + 4 * M and need % 256 == 0
     assert lib.convrot_workspace_bytes(99, M, N, K) == 0
     assert lib.convrot_workspace_bytes(cr.OP_LINEAR_INT8, 0, N, K) == 0
+    # slices of at most 2N tokens: all of M here, 2N = 2048 rows for N = 1024
+    assert lib.convrot_workspace_bytes(cr.OP_LINEAR_INT8_SLICED, M, N, K) == need
+    sliced = lib.convrot_workspace_bytes(cr.OP_LINEAR_INT8_SLICED, M, 1024, K)
+    assert sliced == lib.convrot_workspace_bytes(cr.OP_LINEAR_INT8, 2048, 1024, K)
 
 
 def test_linear_rejects_before_device():

@@ -385,3 +385,32 @@ def test_bounded_wait_timeout_is_reported():
     acc = cr.int8_gemm_s32(torch.from_numpy(a).cuda(), torch.from_numpy(b).cuda())
     np.testing.assert_array_equal(acc.cpu().numpy(), oracle.int8_gemm_acc(a, b))
     cr.check_status()
+
+
+# ---------------------------------------------------------------------------
+# workspace slicing: a smaller workspace processes the tokens in row slices
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+def test_linear_int8_sliced_workspace(dtype):
+    """Slices of at most 2N tokens (the Int8 Compute page's memory bound), of
+    100 tokens, and of a single token give the one-pass result bit for bit."""
+    M, K, N = 700, 1024, 256
+    lin = workloads.Linear("sliced", M, K, N, G=256)
+    inp = workloads.make_layer_inputs(lin, 5, dtype=dtype)
+    rot = cr.Rotation(inp.R)
+    Wq, s_w = cr.quantize_weight(inp.W.cuda(), rot)
+    x, bias = inp.x.cuda(), inp.bias.cuda()
+    full = cr.workspace_bytes(M, N, K)
+    y_ref = cr.linear_int8(x, Wq, s_w, rot, bias, workspace=torch.empty(full, dtype=torch.uint8, device="cuda"))
+    sliced = cr.workspace_bytes(M, N, K, sliced=True)
+    assert sliced < full
+    one_row = cr.workspace_bytes(1, N, K)
+    for nbytes in (sliced, cr.workspace_bytes(100, N, K), one_row):
+        ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+        y = cr.linear_int8(x, Wq, s_w, rot, bias, workspace=ws)
+        torch.cuda.synchronize()
+        assert torch.equal(y.view(torch.int16), y_ref.view(torch.int16)), nbytes
+    with pytest.raises(cr.ConvRotError) as e:
+        cr.linear_int8(x, Wq, s_w, rot, bias,
+                       workspace=torch.empty(one_row - 256, dtype=torch.uint8, device="cuda"))
+    assert e.value.status == cr.WORKSPACE
