@@ -512,6 +512,22 @@ def run_sweep(args):
         out = torch.empty((N, K), dtype=torch.bfloat16, device="cuda")
         t = timed(lambda: cr.dequant_derotate(Wq, s_w, rot, out=out), args.steps)
         dec.append({"G": G, "ms": t, "GBps": 3 * N * K / t / 1e6, "frac_hbm": 3 * N * K / t / 1e6 / hbm_gbs})
+    # few tokens, launched back to back as in a model (chained launches), each
+    # launch on its own weight copy so that the weights (8 x 16.8 MB) stream
+    # from HBM, not L2
+    chained = []
+    rot = cr.Rotation(workloads.sylvester_rotation(256))
+    Ws = [torch.randint(-127, 128, (4096, 4096), dtype=torch.int8, device="cuda") for _ in range(8)]
+    sw1 = torch.tensor([1e-3], device="cuda")
+    for Mc in (1, 16, 128):
+        xq = torch.randint(-127, 128, (Mc, 4096), dtype=torch.int8, device="cuda")
+        st = torch.rand(Mc, device="cuda") * 1e-3
+        y = torch.empty((Mc, 4096), dtype=torch.bfloat16, device="cuda")
+        t = timed(lambda: [cr.int8_gemm(xq, st, W, sw1, None, out=y) for W in Ws], args.steps) / len(Ws)
+        wbytes = Mc * 4096 + 4096 * 4096 + 2 * Mc * 4096
+        chained.append({"M": Mc, "gemm_ms": t, "gemm_GBps": wbytes / t / 1e6,
+                        "gemm_frac_hbm": wbytes / t / 1e6 / hbm_gbs})
+    del Ws
     # per-output-channel weight scales and fp16 activations/outputs, G = 256:
     # the GEMM at M = 8192 and the [12288, 3072] decode
     var = []
@@ -557,6 +573,7 @@ def run_sweep(args):
                       "decode_fp64_tflops": 2.0 * G * N * K / t_d / 1e9})
     print(json.dumps({"sweep": "group_size_and_skinny_M", "linears": rows, "decode_12288x3072": dec,
                       "variants_G256": var, "dense_R_M8192": dense,
+                      "few_tokens_chained_G256": chained,
                       "peaks": {"hbm_gbs": hbm_gbs, "int8_tops": int8_peak}}))
     return 0
 
