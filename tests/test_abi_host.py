@@ -118,3 +118,24 @@ def test_binding_validates_tensors_on_cpu():
         cr.rotate_quant_act(x, None)
     with pytest.raises(ValueError):
         cr.rotate_quant_act(x.to(torch.bfloat16), None)  # not a CUDA tensor
+
+
+def test_header_compiles_as_c_and_links(tmp_path):
+    """include/convrot.h is a C ABI: a C99 program compiled with gcc against the
+    header alone links libconvrot.so and gets the documented argument errors."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("gcc not available")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    lib_dir = os.path.dirname(cr.library_path())
+    exe = str(tmp_path / "abi_smoke")
+    cmd = [gcc, "-std=c99", "-Wall", "-Werror", "-pedantic",
+           os.path.join(root, "tests", "c_abi", "abi_smoke.c"),
+           "-I", os.path.join(root, "include"), "-L", lib_dir, "-lconvrot",
+           "-Wl,-rpath," + lib_dir, "-o", exe]
+    subprocess.run(cmd, check=True, capture_output=True, text=True)
+    res = subprocess.run([exe], capture_output=True, text=True, timeout=120)
+    assert res.returncode == 0, res.stderr
+    assert "c abi ok" in res.stdout
