@@ -119,20 +119,25 @@ __device__ __forceinline__ float widen16(uint16_t v, bool f16) {
   return f16 ? __half2float(__ushort_as_half(v)) : __uint_as_float(static_cast<uint32_t>(v) << 16);
 }
 
+// `valid` (16 or 32) of the 32 columns exist.  Columns 16..31 read their
+// scale and bias through a second base that falls back to columns 0..15 when
+// only 16 exist, so nothing past N is read (those outputs are not stored).
 __device__ __forceinline__ void store_row32(uint16_t* dst, const uint32_t (&r)[32], float scale,
                                             const float* s_w_row, const uint16_t* bias, int valid,
                                             bool f16) {
+  const int hi_base = valid == 32 ? 16 : 0;
   uint32_t w[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
+    const int col = i < 8 ? 2 * i : 2 * i - 16 + hi_base;
     float lo = __int2float_rn(static_cast<int32_t>(r[2 * i]));
     float hi = __int2float_rn(static_cast<int32_t>(r[2 * i + 1]));
-    const float sl = s_w_row ? scale * s_w_row[2 * i] : scale;
-    const float sh = s_w_row ? scale * s_w_row[2 * i + 1] : scale;
+    const float sl = s_w_row ? scale * s_w_row[col] : scale;
+    const float sh = s_w_row ? scale * s_w_row[col + 1] : scale;
     float bl = 0.f, bh = 0.f;
     if (bias) {
-      bl = widen16(bias[2 * i], f16);
-      bh = widen16(bias[2 * i + 1], f16);
+      bl = widen16(bias[col], f16);
+      bh = widen16(bias[col + 1], f16);
     }
     lo = fmaf(lo, sl, bl);
     hi = fmaf(hi, sh, bh);
