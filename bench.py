@@ -42,8 +42,8 @@ INT8_PER_BF16 = 2.0  # nominal dense int8 : bf16 tensor throughput (4.5 : 2.25 P
 # DRAM bytes per launch from ncu (dram__bytes_read.sum + dram__bytes_write.sum),
 # averaged over the three GEMM launches of one Z-Image step, valid only for the
 # kernel source they were taken on (first 16 hex digits of its sha256).
-NCU_TRAFFIC = {"int8_gemm_tcgen05": (121.19e6 + 100.52e6 + 152.26e6) / 3}
-NCU_TRAFFIC_SOURCE_SHA = {"int8_gemm_tcgen05": "43b6e5068503ed91"}
+NCU_TRAFFIC = {"int8_gemm_tcgen05": (120.19e6 + 101.99e6 + 151.16e6) / 3}
+NCU_TRAFFIC_SOURCE_SHA = {"int8_gemm_tcgen05": "b5f9eeca52952e70"}
 
 
 def source_sha(rel: str) -> str:
