@@ -5,11 +5,18 @@
 //   D[n, m] = sum_k Wq[n, k] * xq[m, k]   (n: 128 weight rows per CTA, m: NT >= M tokens)
 //
 // K is split over a cluster of S CTAs (S <= 8) that share one 128-row block of
-// the weight; each CTA accumulates its K range in TMEM, parks the int32
-// partial in its shared memory, and after a cluster barrier every CTA sums
-// the S partials of its share of the rows through distributed shared memory
-// and applies the rescale/bias epilogue (or stores int32).  No global
-// scratch.  Same warp roles and bounded waits as the main GEMM.
+// the weight; each CTA accumulates its K range in TMEM and parks the int32
+// partial in its shared memory.  After a cluster barrier every CTA pushes the
+// rows each peer finishes into that peer's shared memory with one bulk copy
+// per peer (completed on the peer's mbarrier), then sums the S partials of its
+// own 128 / S rows from local shared memory and applies the rescale/bias
+// epilogue (or stores int32).  No global scratch.  Same warp roles and bounded
+// waits as the main GEMM.
+//
+// Bulk copies rather than per-thread loads through the cluster window: with
+// every thread pulling 16-byte pieces of its peers' partials the reduction
+// ran at a few bytes per clock per SM and took half of the kernel at 128
+// tokens; keeping more such loads in flight made it slower still.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -49,14 +56,18 @@ struct SkinnyCfg {
   static constexpr int kAStage = kRows * kBK;
   static constexpr int kBStage = NT * kBK;
   static constexpr int kStageBytes = kAStage + kBStage;
+  // epilogue factors staged during the mainloop: s_tok of the NT tokens, s_w
+  // and bias of the block's rows (f32)
+  static constexpr int kEpiBytes = (NT + 2 * kRows) * 4;
   // as many stages as fit (a CTA's whole K range in flight at once); the int32
   // partial reuses the ring once the mainloop has drained it
-  static constexpr int kFit = (232448 - 1024 - 256) / kStageBytes;
+  static constexpr int kFit = (232448 - 1024 - 256 - kEpiBytes) / kStageBytes;
   static constexpr int kStages = kFit > 12 ? 12 : kFit;
   static constexpr int kPartStride = NT + 4;  // int32 per partial row (padded: no bank conflicts)
   static constexpr int kPartBytes = kRows * kPartStride * 4;
-  static_assert(kPartBytes <= kStages * kStageBytes, "partial must fit in the ring");
-  static constexpr size_t kSmem = 1024 + kStages * kStageBytes + 256;
+  // the partial and, after it, the slices the peers push (one per rank)
+  static_assert(2 * kPartBytes <= kStages * kStageBytes, "partial and slices must fit in the ring");
+  static constexpr size_t kSmem = 1024 + kStages * kStageBytes + 256 + kEpiBytes;
   static constexpr uint32_t kTmemCols = NT < 32 ? 32 : NT;
   static constexpr uint32_t kIdesc = ptx::idesc_i8(kRows, NT);
 };
@@ -66,6 +77,7 @@ struct SkinnyBars {
   uint64_t full[STAGES];
   uint64_t empty[STAGES];
   uint64_t acc_full;
+  uint64_t recv_full;  // the peers' slices have landed
   uint32_t tmem_base;
   uint32_t abort_flag;
 };
@@ -82,8 +94,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sA = smem;
   uint8_t* sB = smem + kStages * C::kAStage;
   int32_t* part = reinterpret_cast<int32_t*>(smem);  // after the mainloop only
+  int32_t* recv = part + kRows * C::kPartStride;     // [splits][rows][kPartStride]
   auto* bars = reinterpret_cast<SkinnyBars<kStages>*>(smem + kStages * C::kStageBytes);
   volatile uint32_t* abort_flag = &bars->abort_flag;
+  float* ep_tok = reinterpret_cast<float*>(smem + kStages * C::kStageBytes + 256);  // [NT]
+  float* ep_sw = ep_tok + NT;      // [rows], this CTA's share of the block
+  float* ep_bias = ep_sw + kRows;  // [rows]
 
   const int warp = threadIdx.x >> 5;
   const uint32_t lane = threadIdx.x & 31;
@@ -91,6 +107,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int block = static_cast<int>(blockIdx.x) / p.splits;  // 128-row block of the weight
   const int kb0 = static_cast<int>(rank) * p.kb_per_split;
   const int kb1 = min(p.num_kb, kb0 + p.kb_per_split);
+  // after the split-K reduction this CTA finishes rows [r0, r0 + rows) of the block
+  const int rows = kRows / p.splits;
+  const int r0 = static_cast<int>(rank) * rows;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -98,6 +117,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::mbar_init(&bars->empty[s], 1);
     }
     ptx::mbar_init(&bars->acc_full, 1);
+    ptx::mbar_init(&bars->recv_full, 1);
     bars->abort_flag = 0;
     ptx::fence_mbarrier_init();
     ptx::tma_prefetch_desc(&tmW);
@@ -162,6 +182,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     // publishes the accumulator once every MMA issued above has completed
     ptx::mma_commit(&bars->acc_full);
   } else if (warp >= 2) {
+    // ------------------------------------------------------------ epilogue factors
+    // read while the mainloop streams the weight, so the reduction below
+    // touches no global memory before its stores
+    if (!p.out_s32) {
+      const int t = static_cast<int>(threadIdx.x) - 64;
+      for (int m = t; m < NT; m += kThreads - 64) ep_tok[m] = m < p.M ? p.s_tok[m] : 0.f;
+      for (int r = t; r < rows; r += kThreads - 64) {
+        const int64_t n = static_cast<int64_t>(block) * kRows + r0 + r;
+        float sw = 0.f, bn = 0.f;
+        if (n < p.N) {
+          sw = p.per_channel_scale ? p.s_w[n] : p.s_w[0];
+          if (p.bias) {
+            bn = p.out_f16 ? __half2float(__ushort_as_half(p.bias[n]))
+                           : __uint_as_float(static_cast<uint32_t>(p.bias[n]) << 16);
+          }
+        }
+        ep_sw[r] = sw;
+        ep_bias[r] = bn;
+      }
+    }
     // ------------------------------------------------------------ partial -> shared memory
     const int quarter = warp & 3;
     const int row = quarter * 32 + static_cast<int>(lane);
@@ -197,42 +237,61 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   // ---------------------------------------------------------------- split-K reduction
+  const uint32_t slice_words = static_cast<uint32_t>(rows * C::kPartStride);
+  if (warp >= 2) ptx::fence_proxy_async_smem();  // the partial, for the bulk copies below
+  if (threadIdx.x == 0 && p.splits > 1) {
+    // armed before the barrier: no peer pushes before every CTA has passed it
+    ptx::mbar_arrive_expect_tx(&bars->recv_full, static_cast<uint32_t>(p.splits - 1) * slice_words * 4u);
+  }
   ptx::tc_fence_before();
-  ptx::cluster_sync();  // every CTA's partial is in its shared memory
+  ptx::cluster_sync();  // every CTA's partial (and the staged factors) in shared memory
+  if (p.splits > 1) {
+    // push rank o's rows of this CTA's partial into slot [rank] of rank o
+    if (threadIdx.x == 0) {
+      for (int o = 0; o < p.splits; ++o) {
+        if (o == static_cast<int>(rank)) continue;
+        ptx::bulk_copy_to_peer(
+            ptx::mapa_shared(ptx::smem_u32(recv + rank * slice_words), static_cast<uint32_t>(o)),
+            ptx::smem_u32(part + o * slice_words), slice_words * 4u,
+            ptx::mapa_shared(ptx::smem_u32(&bars->recv_full), static_cast<uint32_t>(o)));
+      }
+    }
+    if (!ptx::mbar_wait(&bars->recv_full, 0, ptx::globaltimer_ns() + kWaitNs) && lane == 0) {
+      atomicOr(p.status, 1u);
+    }
+  }
+  // every copy into this CTA has landed; once all ranks have arrived, every
+  // copy out of this CTA has too, and its shared memory may be released
+  __syncwarp();
+  ptx::cluster_arrive();
   {
-    // this CTA finishes rows [r0, r0 + rows) of the block, for all tokens
-    const int rows = kRows / p.splits;
-    const int r0 = static_cast<int>(rank) * rows;
-    const uint32_t part_local = ptx::smem_u32(part);
-    const int items = rows * (NT / 4);  // (row, 4 tokens) items
+    // (row, 4 tokens) items; consecutive threads take consecutive weight rows
+    const int items = rows * (NT / 4);
     for (int it = threadIdx.x; it < items; it += kThreads) {
-      const int rr = r0 + it % rows;   // consecutive threads -> consecutive weight rows
+      const int r = it % rows;
       const int m4 = (it / rows) * 4;  // first of 4 tokens
-      int32_t acc[4] = {0, 0, 0, 0};
-      const uint32_t off = static_cast<uint32_t>((rr * C::kPartStride + m4) * 4);
+      int4 acc = *reinterpret_cast<const int4*>(part + (r0 + r) * C::kPartStride + m4);
       for (int s = 0; s < p.splits; ++s) {
-        const uint4 v = ptx::ld_cluster_v4(ptx::mapa_shared(part_local + off, static_cast<uint32_t>(s)));
-        acc[0] += static_cast<int32_t>(v.x);
-        acc[1] += static_cast<int32_t>(v.y);
-        acc[2] += static_cast<int32_t>(v.z);
-        acc[3] += static_cast<int32_t>(v.w);
+        if (s == static_cast<int>(rank)) continue;
+        const int4 v = *reinterpret_cast<const int4*>(recv + s * slice_words + r * C::kPartStride + m4);
+        acc.x += v.x;
+        acc.y += v.y;
+        acc.z += v.z;
+        acc.w += v.w;
       }
-      const int64_t n = static_cast<int64_t>(block) * kRows + rr;
+      const int32_t a4[4] = {acc.x, acc.y, acc.z, acc.w};
+      const int64_t n = static_cast<int64_t>(block) * kRows + r0 + r;
       if (n >= p.N) continue;
-      const float sw = p.out_s32 ? 0.f : (p.per_channel_scale ? p.s_w[n] : p.s_w[0]);
-      float bn = 0.f;
-      if (!p.out_s32 && p.bias) {
-        bn = p.out_f16 ? __half2float(__ushort_as_half(p.bias[n]))
-                       : __uint_as_float(static_cast<uint32_t>(p.bias[n]) << 16);
-      }
+      const float sw = p.out_s32 ? 0.f : ep_sw[r];
+      const float bn = p.out_s32 ? 0.f : ep_bias[r];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int64_t m = m4 + j;
         if (m >= p.M) break;
         if (p.out_s32) {
-          static_cast<int32_t*>(p.out)[m * p.N + n] = acc[j];
+          static_cast<int32_t*>(p.out)[m * p.N + n] = a4[j];
         } else {
-          const float y = fmaf(__int2float_rn(acc[j]), p.s_tok[m] * sw, bn);
+          const float y = fmaf(__int2float_rn(a4[j]), ep_tok[m] * sw, bn);
           uint16_t bits;
           if (p.out_f16) {
             bits = __half_as_ushort(__float2half_rn(y));
@@ -245,7 +304,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   }
-  ptx::cluster_sync();  // peers' partials stay alive until every CTA has read them
+  __syncwarp();
+  ptx::cluster_wait();
   if (warp == 1) {
     __syncwarp();
     ptx::tc_fence_after();

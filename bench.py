@@ -519,7 +519,7 @@ def run_sweep(args):
     rot = cr.Rotation(workloads.sylvester_rotation(256))
     Ws = [torch.randint(-127, 128, (4096, 4096), dtype=torch.int8, device="cuda") for _ in range(8)]
     sw1 = torch.tensor([1e-3], device="cuda")
-    for Mc in (1, 16, 128):
+    for Mc in (1, 16, 64, 128):
         xq = torch.randint(-127, 128, (Mc, 4096), dtype=torch.int8, device="cuda")
         st = torch.rand(Mc, device="cuda") * 1e-3
         y = torch.empty((Mc, 4096), dtype=torch.bfloat16, device="cuda")

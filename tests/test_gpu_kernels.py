@@ -56,7 +56,7 @@ def _codes(rng, shape):
 # ---------------------------------------------------------------------------
 GEMM_SHAPES = [
     (1, 16, 16), (7, 144, 64), (128, 256, 128), (129, 272, 144), (257, 512, 1024),
-    (300, 1024, 3840), (64, 1024, 1024), (1000, 528, 2048), (33, 4096, 256),
+    (300, 1024, 3840), (64, 1024, 1024), (1000, 528, 2048), (33, 4096, 256), (97, 1008, 4096),
 ]
 
 
@@ -124,7 +124,7 @@ def _assert_epilogue_close(y_gpu, acc, s_tok, s_w, bias):
 
 @pytest.mark.parametrize("M,N,K,with_bias,per_channel", [
     (64, 1024, 1024, True, False), (129, 272, 144, False, False), (7, 144, 64, True, True),
-    (257, 512, 256, True, True),
+    (257, 512, 256, True, True), (100, 1008, 2048, True, True),
 ])
 def test_int8_gemm_epilogue(M, N, K, with_bias, per_channel):
     rng = np.random.default_rng(M + N + K)
