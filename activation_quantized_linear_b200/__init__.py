@@ -15,8 +15,12 @@ Entry points (same names as the C ABI, without the `convrot_` prefix; the
     int8_gemm_s32(xq, Wq)                    -> acc (int32)
     linear_int8(x, Wq, s_w, rot, bias)       -> y (x's dtype)
     linear_int8_noalloc(x, Wq, s_w, rot, bias) -> y (bf16; the library's static scratch)
+    dense_linear(x, W, bias)                 -> y (the default path's 16-bit matmul)
+    linear_dequant(x, Wq, s_w, rot, bias)    -> y (the default path: decode, then dense_linear)
+    linear_checked(x, Wq, s_w, rot, bias)    -> (y, path) (int8 compute, first call checked)
+    check_state(device), check_reset(), check_set_min_cosine(t), check_min_cosine()
     workspace_bytes(M, N, K), check_status(), selftest_wait_timeout(ms)
-    ConvRotLinear(W, R, bias)                 the layer: forward (int8 compute), decode_weight
+    ConvRotLinear(W, R, bias, mode)           the layer: forward, decode_weight
 """
 
 from __future__ import annotations
@@ -33,11 +37,14 @@ __all__ = [
     "ConvRotError", "Rotation", "quantize_weight", "dequant_derotate", "rotate_quant_act",
     "int8_gemm", "int8_gemm_s32", "linear_int8", "workspace_bytes", "check_status",
     "device_supported", "library_path", "ConvRotLinear", "linear_int8_noalloc",
-    "noalloc_scratch_bytes", "selftest_wait_timeout",
+    "noalloc_scratch_bytes", "selftest_wait_timeout", "dense_linear", "linear_dequant",
+    "linear_checked", "check_state", "check_reset", "check_set_min_cosine", "check_min_cosine",
 ]
 
 OK, INVALID_ARG, UNSUPPORTED, CUDA, WORKSPACE, TIMEOUT, ALIGNMENT = range(7)
-OP_LINEAR_INT8, OP_LINEAR_INT8_SLICED = 1, 2
+OP_LINEAR_INT8, OP_LINEAR_INT8_SLICED, OP_LINEAR_DEQUANT, OP_LINEAR_CHECKED = 1, 2, 3, 4
+PATH_INT8, PATH_DEQUANT = 1, 2
+CHECK_ROWS = 256
 STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "CUDA", 4: "WORKSPACE",
                 5: "TIMEOUT", 6: "ALIGNMENT"}
 
@@ -83,7 +90,17 @@ def _load() -> ctypes.CDLL:
         "convrot_rotate_quant_act_f16": ([vp, i64, i64, vp, vp, vp, vp], i32),
         "convrot_int8_gemm_f16": ([vp, vp, vp, vp, i64, vp, i64, i64, i64, vp, vp], i32),
         "convrot_linear_int8_f16": ([vp, i64, i64, i64, vp, vp, vp, i64, vp, vp, vp, sz, vp], i32),
+        "convrot_check_state": ([i32, ctypes.POINTER(i32), ctypes.POINTER(i32)], i32),
+        "convrot_check_reset": ([], None),
+        "convrot_check_set_min_cosine": ([ctypes.c_double], i32),
+        "convrot_check_min_cosine": ([], ctypes.c_double),
     }
+    for f in ("", "_f16"):
+        sigs["convrot_dense_linear" + f] = ([vp, i64, i64, i64, vp, vp, vp, vp], i32)
+        sigs["convrot_linear_dequant" + f] = (
+            [vp, i64, i64, i64, vp, vp, vp, i64, vp, vp, vp, sz, vp], i32)
+        sigs["convrot_linear_checked" + f] = (
+            [vp, i64, i64, i64, vp, vp, vp, i64, vp, vp, vp, sz, ctypes.POINTER(i32), vp], i32)
     for name, (args, res) in sigs.items():
         fn = getattr(lib, name)
         fn.argtypes = args
@@ -263,11 +280,20 @@ def int8_gemm_s32(xq: torch.Tensor, Wq: torch.Tensor, out: torch.Tensor | None =
     return out
 
 
-def workspace_bytes(M: int, N: int, K: int, sliced: bool = False) -> int:
+def workspace_bytes(M: int, N: int, K: int, sliced: bool = False, op: int | None = None) -> int:
     """Workspace of linear_int8 for all M tokens at once, or (sliced=True) for
-    slices of at most 2N tokens; any size down to one row works."""
-    op = OP_LINEAR_INT8_SLICED if sliced else OP_LINEAR_INT8
+    slices of at most 2N tokens; any size down to one row works.  `op` names
+    another operation (OP_LINEAR_DEQUANT, OP_LINEAR_CHECKED)."""
+    if op is None:
+        op = OP_LINEAR_INT8_SLICED if sliced else OP_LINEAR_INT8
     return int(_lib.convrot_workspace_bytes(op, M, N, K))
+
+
+def _workspace(workspace: torch.Tensor | None, need: int, device) -> torch.Tensor:
+    if workspace is None:
+        return torch.empty(max(need, 1), dtype=torch.uint8, device=device)
+    _need(workspace, "workspace", torch.uint8, 1)
+    return workspace
 
 
 def linear_int8(x: torch.Tensor, Wq: torch.Tensor, s_w: torch.Tensor, rot: Rotation,
@@ -312,6 +338,85 @@ def linear_int8_noalloc(x: torch.Tensor, Wq: torch.Tensor, s_w: torch.Tensor, ro
     return out
 
 
+def dense_linear(x: torch.Tensor, W: torch.Tensor, bias: torch.Tensor | None = None,
+                 out: torch.Tensor | None = None) -> torch.Tensor:
+    """The default path's matmul: y = x W^T + bias, x, W, bias and y in one
+    16-bit float format, fp32 accumulation on the tensor cores."""
+    _need16(x, "x", 2)
+    _need(W, "W", x.dtype, 2)
+    if bias is not None:
+        _need(bias, "bias", x.dtype, 1)
+    M, K = x.shape
+    N = W.shape[0]
+    if W.shape[1] != K:
+        raise ValueError(f"W has {W.shape[1]} input features, x has {K}")
+    out = torch.empty((M, N), dtype=x.dtype, device=x.device) if out is None else out
+    _need(out, "out", x.dtype, 2)
+    _check(_fn("convrot_dense_linear", x.dtype)(_ptr(x), M, K, N, _ptr(W), _ptr(bias), _ptr(out),
+                                                 _stream()))
+    return out
+
+
+def _linear_args(x, Wq, s_w, bias, out):
+    _need16(x, "x", 2)
+    _need(Wq, "Wq", torch.int8, 2)
+    _need(s_w, "s_w", torch.float32, 1)
+    if bias is not None:
+        _need(bias, "bias", x.dtype, 1)
+    M, K = x.shape
+    N = Wq.shape[0]
+    out = torch.empty((M, N), dtype=x.dtype, device=x.device) if out is None else out
+    _need(out, "out", x.dtype, 2)
+    return M, K, N, out
+
+
+def linear_dequant(x: torch.Tensor, Wq: torch.Tensor, s_w: torch.Tensor, rot: Rotation,
+                   bias: torch.Tensor | None = None, out: torch.Tensor | None = None,
+                   workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """The default path: decode the weight (into the workspace), then dense_linear."""
+    M, K, N, out = _linear_args(x, Wq, s_w, bias, out)
+    workspace = _workspace(workspace, workspace_bytes(M, N, K, op=OP_LINEAR_DEQUANT), x.device)
+    _check(_fn("convrot_linear_dequant", x.dtype)(
+        _ptr(x), M, K, N, rot.handle, _ptr(Wq), _ptr(s_w), s_w.numel(), _ptr(bias), _ptr(out),
+        _ptr(workspace), workspace.numel(), _stream()))
+    return out
+
+
+def linear_checked(x: torch.Tensor, Wq: torch.Tensor, s_w: torch.Tensor, rot: Rotation,
+                   bias: torch.Tensor | None = None, out: torch.Tensor | None = None,
+                   workspace: torch.Tensor | None = None) -> tuple[torch.Tensor, int]:
+    """The int8-compute forward whose first call per (layer shape, token bucket)
+    is checked against the default path; returns (y, PATH_INT8 or PATH_DEQUANT)."""
+    M, K, N, out = _linear_args(x, Wq, s_w, bias, out)
+    workspace = _workspace(workspace, workspace_bytes(M, N, K, op=OP_LINEAR_CHECKED), x.device)
+    path = ctypes.c_int(0)
+    _check(_fn("convrot_linear_checked", x.dtype)(
+        _ptr(x), M, K, N, rot.handle, _ptr(Wq), _ptr(s_w), s_w.numel(), _ptr(bias), _ptr(out),
+        _ptr(workspace), workspace.numel(), ctypes.byref(path), _stream()))
+    return out, path.value
+
+
+def check_state(device: int | None = None) -> tuple[bool, int]:
+    """(latched onto the default path, number of checked keys) of a CUDA device."""
+    dev = torch.cuda.current_device() if device is None else int(device)
+    latched, keys = ctypes.c_int(0), ctypes.c_int(0)
+    _check(_lib.convrot_check_state(dev, ctypes.byref(latched), ctypes.byref(keys)))
+    return bool(latched.value), int(keys.value)
+
+
+def check_reset() -> None:
+    """Forget every checked key and latch (as a process restart would)."""
+    _lib.convrot_check_reset()
+
+
+def check_set_min_cosine(threshold: float) -> None:
+    _check(_lib.convrot_check_set_min_cosine(float(threshold)))
+
+
+def check_min_cosine() -> float:
+    return float(_lib.convrot_check_min_cosine())
+
+
 def noalloc_scratch_bytes() -> int:
     return int(_lib.convrot_noalloc_scratch_bytes())
 
@@ -331,15 +436,25 @@ def selftest_wait_timeout(limit_ms: int = 20) -> None:
 class ConvRotLinear:
     """A ConvRot int8_tensorwise linear: int8 weight, per-tensor scale, rotation R.
 
-    `forward` runs the int8-compute path in the input's format (bf16 or fp16;
-    the bias, if any, must match it); `decode_weight` the default path's weight
-    decode (dequantize + derotate) to W's format unless `dtype` says otherwise."""
+    `forward` runs in the input's format (bf16 or fp16; the bias, if any, must
+    match it) on the path `mode` names: "int8" (int8 compute), "dequant" (the
+    default path: decode the weight, then a 16-bit matmul) or "checked" (int8
+    compute whose first call per layer shape and token bucket is checked
+    against the default path, falling back to it on a mismatch).
+    `decode_weight` is the default path's weight decode (dequantize +
+    derotate), to W's format unless `dtype` says otherwise."""
 
-    def __init__(self, W: torch.Tensor, R, bias: torch.Tensor | None = None):
+    MODES = ("int8", "dequant", "checked")
+
+    def __init__(self, W: torch.Tensor, R, bias: torch.Tensor | None = None, mode: str = "int8"):
+        if mode not in self.MODES:
+            raise ValueError(f"mode must be one of {self.MODES}, got {mode!r}")
         self.rotation = R if isinstance(R, Rotation) else Rotation(R)
         self.Wq, self.s_w = quantize_weight(W, self.rotation)
         self.dtype = W.dtype
         self.bias = bias
+        self.mode = mode
+        self.last_path = None
         self._ws = None
 
     @property
@@ -357,10 +472,19 @@ class ConvRotLinear:
 
     def forward(self, x: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
         M = x.shape[0]
-        need = workspace_bytes(M, self.out_features, self.in_features)
+        op = {"int8": OP_LINEAR_INT8, "dequant": OP_LINEAR_DEQUANT,
+              "checked": OP_LINEAR_CHECKED}[self.mode]
+        need = workspace_bytes(M, self.out_features, self.in_features, op=op)
         if self._ws is None or self._ws.numel() < need:
             self._ws = torch.empty(max(need, 1), dtype=torch.uint8, device=x.device)
-        return linear_int8(x, self.Wq, self.s_w, self.rotation, self.bias, out=out,
-                           workspace=self._ws)
+        args = (x, self.Wq, self.s_w, self.rotation, self.bias)
+        if self.mode == "int8":
+            self.last_path = PATH_INT8
+            return linear_int8(*args, out=out, workspace=self._ws)
+        if self.mode == "dequant":
+            self.last_path = PATH_DEQUANT
+            return linear_dequant(*args, out=out, workspace=self._ws)
+        y, self.last_path = linear_checked(*args, out=out, workspace=self._ws)
+        return y
 
     __call__ = forward

@@ -387,11 +387,66 @@ convrot_status convrot_int8_gemm_s32(const int8_t* xq, const int8_t* Wq, int64_t
   return gemm_common(xq, nullptr, Wq, nullptr, 1, nullptr, M, N, K, acc, true, false, stream);
 }
 
+static convrot_status dense_linear_impl(const uint16_t* x, bool f16, int64_t M, int64_t K,
+                                        int64_t N, const uint16_t* W, const uint16_t* bias,
+                                        uint16_t* y, convrot_stream_t stream) {
+  convrot_status s = check_gemm_shape(M, N, K);
+  if (s != CONVROT_OK) return s;
+  if (M == 0) return CONVROT_OK;
+  CHECK_PTR(x);
+  CHECK_PTR(W);
+  CHECK_PTR(y);
+  if (bias != nullptr && !aligned16(bias)) {
+    return fail(CONVROT_ERR_ALIGNMENT, "bias is not 16-byte aligned");
+  }
+  int dev = -1;
+  s = current_device(&dev);
+  if (s != CONVROT_OK) return s;
+  convrot::GemmArgs a;
+  a.A = nullptr;
+  a.B = nullptr;
+  a.s_tok = nullptr;
+  a.s_w = nullptr;
+  a.s_w_len = 1;
+  a.bias = bias;
+  a.out = y;
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.out_s32 = false;
+  a.out_f16 = f16;
+  a.ops16 = true;
+  a.A16 = x;
+  a.B16 = W;
+  cudaError_t e = convrot::launch_gemm16(a, as_stream(stream));
+  if (e == cudaErrorInvalidValue) {
+    return fail(CONVROT_ERR_CUDA, "dense_linear: TMA descriptor encoding failed");
+  }
+  return launched(e, "dense_linear launch");
+}
+
+convrot_status convrot_dense_linear(const convrot_bf16* x, int64_t M, int64_t K, int64_t N,
+                                    const convrot_bf16* W, const convrot_bf16* bias,
+                                    convrot_bf16* y, convrot_stream_t stream) {
+  return dense_linear_impl(x, false, M, K, N, W, bias, y, stream);
+}
+
+convrot_status convrot_dense_linear_f16(const convrot_f16* x, int64_t M, int64_t K, int64_t N,
+                                        const convrot_f16* W, const convrot_f16* bias,
+                                        convrot_f16* y, convrot_stream_t stream) {
+  return dense_linear_impl(x, true, M, K, N, W, bias, y, stream);
+}
+
 // Workspace of a slice of `rows` tokens: the int8 codes, then (256-byte
 // aligned) the per-token scales.
 static size_t slice_bytes(int64_t rows, int64_t K) {
   return align256(static_cast<size_t>(rows) * static_cast<size_t>(K)) +
          align256(sizeof(float) * static_cast<size_t>(rows));
+}
+
+// The decoded weight of the default path.
+static size_t decoded_weight_bytes(int64_t N, int64_t K) {
+  return align256(2 * static_cast<size_t>(N) * static_cast<size_t>(K));
 }
 
 size_t convrot_workspace_bytes(int op, int64_t M, int64_t N, int64_t K) {
@@ -401,7 +456,52 @@ size_t convrot_workspace_bytes(int op, int64_t M, int64_t N, int64_t K) {
     const int64_t rows = M < 2 * N ? M : 2 * N;
     return slice_bytes(rows, K);
   }
+  if (op == CONVROT_OP_LINEAR_DEQUANT) return decoded_weight_bytes(N, K);
+  if (op == CONVROT_OP_LINEAR_CHECKED) {
+    // the int8 forward's codes, or (reusing the same bytes once it is done)
+    // the decoded weight, the default path's rows under check and the sums
+    const int64_t rows = M < CONVROT_CHECK_ROWS ? M : CONVROT_CHECK_ROWS;
+    const size_t check = decoded_weight_bytes(N, K) +
+                         align256(2 * static_cast<size_t>(rows) * static_cast<size_t>(N)) + 256;
+    const size_t fwd = slice_bytes(M, K);
+    return fwd > check ? fwd : check;
+  }
   return 0;
+}
+
+static convrot_status linear_dequant_impl(const uint16_t* x, bool f16, int64_t M, int64_t K,
+                                          int64_t N, convrot_rotation_t R, const int8_t* Wq,
+                                          const float* s_w, int64_t s_w_len, const uint16_t* bias,
+                                          uint16_t* y, void* ws, size_t ws_bytes,
+                                          convrot_stream_t stream) {
+  convrot_status s = check_gemm_shape(M, N, K);
+  if (s != CONVROT_OK) return s;
+  if (M == 0) return CONVROT_OK;
+  const size_t need = decoded_weight_bytes(N, K);
+  if (ws == nullptr || ws_bytes < need) {
+    return fail(CONVROT_ERR_WORKSPACE, "workspace of %zu bytes given, %zu needed", ws_bytes, need);
+  }
+  if (reinterpret_cast<uintptr_t>(ws) & 255u) {
+    return fail(CONVROT_ERR_WORKSPACE, "workspace is not 256-byte aligned");
+  }
+  uint16_t* W_hat = static_cast<uint16_t*>(ws);
+  s = dequant_derotate_impl(Wq, s_w, s_w_len, N, K, R, W_hat, f16, stream);
+  if (s != CONVROT_OK) return s;
+  return dense_linear_impl(x, f16, M, K, N, W_hat, bias, y, stream);
+}
+
+convrot_status convrot_linear_dequant(const convrot_bf16* x, int64_t M, int64_t K, int64_t N,
+                                      convrot_rotation_t R, const int8_t* Wq, const float* s_w,
+                                      int64_t s_w_len, const convrot_bf16* bias, convrot_bf16* y,
+                                      void* ws, size_t ws_bytes, convrot_stream_t stream) {
+  return linear_dequant_impl(x, false, M, K, N, R, Wq, s_w, s_w_len, bias, y, ws, ws_bytes, stream);
+}
+
+convrot_status convrot_linear_dequant_f16(const convrot_f16* x, int64_t M, int64_t K, int64_t N,
+                                          convrot_rotation_t R, const int8_t* Wq, const float* s_w,
+                                          int64_t s_w_len, const convrot_f16* bias, convrot_f16* y,
+                                          void* ws, size_t ws_bytes, convrot_stream_t stream) {
+  return linear_dequant_impl(x, true, M, K, N, R, Wq, s_w, s_w_len, bias, y, ws, ws_bytes, stream);
 }
 
 static convrot_status linear_int8_impl(const uint16_t* x, bool f16, int64_t M, int64_t K,

@@ -21,6 +21,9 @@
 // commits signal both CTAs' barriers.  A pair moves 2/3 of the operand bytes
 // per MMA that two single CTAs would.  (Up to 128 tokens take the swap-AB
 // kernel in int8_gemm_skinny.cu instead.)
+// The same pipeline with 16-bit operands (kind::f16, fp32 accumulator, no
+// scales: y = f16(acc + bias)) is the dense linear of the default path, which
+// multiplies by the decoded weight (gemm16_tcgen05).
 // Every mbarrier wait is bounded by the global timer.  A wait that runs out
 // records CONVROT_ERR_TIMEOUT in the device status word; the CTA then stops
 // issuing work, drains what it issued and frees its TMEM before returning.
@@ -40,18 +43,22 @@ namespace {
 
 constexpr int BM = 128;       // accumulator rows per CTA (TMEM lanes)
 constexpr int BN = 256;       // accumulator columns per tile
-constexpr int BK = 128;       // bytes = int8 elements per stage; one 128-byte swizzle row
-constexpr int UMMA_K = 32;
+constexpr int BK = 128;       // bytes per operand row per stage; one 128-byte swizzle row
+constexpr int UMMA_K = 32;    // bytes of K per MMA (32 int8 or 16 16-bit elements)
 constexpr int A_STAGE = BM * BK;
-constexpr int ACC_COLS = BN;  // int32 accumulator columns per tile
+constexpr int ACC_COLS = BN;  // 32-bit accumulator columns per tile
 constexpr uint32_t TMEM_COLS = 2 * ACC_COLS;
 constexpr int kThreads = 192;
 constexpr int kEpiWarps = 4;
 constexpr uint64_t kWaitNs = 1000000000ull;  // 1 s per wait
 
+// Operand kinds: int8 (int32 accumulator, ConvRot epilogue), or bf16 / fp16
+// (fp32 accumulator, bias only).
+constexpr int kKindI8 = 0, kKindBF16 = 1, kKindF16 = 2;
+
 // A cluster of two CTAs per tile of 256 x 256 (cta_group::2); each CTA loads
 // its 128 rows of A and its 128 rows of B per stage, 6 stages, and only the
-// even CTA issues the MMAs.
+// even CTA issues the MMAs.  The geometry is in bytes, the same for every kind.
 struct Cfg {
   static constexpr int kBRows = BN / 2;  // B rows loaded per CTA
   static constexpr int kBStage = kBRows * BK;
@@ -59,9 +66,16 @@ struct Cfg {
   static constexpr int kStages = 6;
   static constexpr int kTileM = 2 * BM;
   static constexpr size_t kSmem = 1024 + kStages * kStageBytes + 256;
-  static constexpr uint32_t kIdesc = ptx::idesc_i8(kTileM, BN);
   // bytes that complete one stage on the leader's full barrier (both CTAs' loads)
   static constexpr uint32_t kTxBytes = 2 * kStageBytes;
+};
+
+template <int kKind>
+struct KindCfg {
+  static constexpr uint32_t kIdesc = kKind == kKindI8
+                                         ? ptx::idesc_i8(Cfg::kTileM, BN)
+                                         : ptx::idesc_f16(Cfg::kTileM, BN, kKind == kKindF16);
+  static constexpr int kStageK = kKind == kKindI8 ? BK : BK / 2;  // K elements per stage
 };
 
 struct Params {
@@ -114,7 +128,8 @@ __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity) {
 }
 
 // 32 outputs of one row: y = f16(float(acc) * scale [* s_w_row] + bias), in bf16
-// or fp16 (f16), rounded once from the fp32 FMA.
+// or fp16 (f16), rounded once from the fp32 FMA.  The accumulator columns hold
+// int32 (kF32Acc = false) or fp32 (true: scale is 1, so y = f16(acc + bias)).
 __device__ __forceinline__ float widen16(uint16_t v, bool f16) {
   return f16 ? __half2float(__ushort_as_half(v)) : __uint_as_float(static_cast<uint32_t>(v) << 16);
 }
@@ -122,6 +137,7 @@ __device__ __forceinline__ float widen16(uint16_t v, bool f16) {
 // `valid` (16 or 32) of the 32 columns exist.  Columns 16..31 read their
 // scale and bias through a second base that falls back to columns 0..15 when
 // only 16 exist, so nothing past N is read (those outputs are not stored).
+template <bool kF32Acc>
 __device__ __forceinline__ void store_row32(uint16_t* dst, const uint32_t (&r)[32], float scale,
                                             const float* s_w_row, const uint16_t* bias, int valid,
                                             bool f16) {
@@ -130,8 +146,9 @@ __device__ __forceinline__ void store_row32(uint16_t* dst, const uint32_t (&r)[3
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
     const int col = i < 8 ? 2 * i : 2 * i - 16 + hi_base;
-    float lo = __int2float_rn(static_cast<int32_t>(r[2 * i]));
-    float hi = __int2float_rn(static_cast<int32_t>(r[2 * i + 1]));
+    float lo = kF32Acc ? __uint_as_float(r[2 * i]) : __int2float_rn(static_cast<int32_t>(r[2 * i]));
+    float hi = kF32Acc ? __uint_as_float(r[2 * i + 1])
+                       : __int2float_rn(static_cast<int32_t>(r[2 * i + 1]));
     const float sl = s_w_row ? scale * s_w_row[col] : scale;
     const float sh = s_w_row ? scale * s_w_row[col + 1] : scale;
     float bl = 0.f, bh = 0.f;
@@ -166,10 +183,11 @@ __device__ __forceinline__ void store_s32_row32(int32_t* dst, const uint32_t (&r
   }
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
-    int8_gemm_tcgen05(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                      const Params p) {
+template <int kKind>
+__device__ __forceinline__ void gemm_pair(const CUtensorMap& tmA, const CUtensorMap& tmB,
+                                          const Params& p) {
   using C = Cfg;
+  using KC = KindCfg<kKind>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -232,8 +250,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         if (leader) ptx::mbar_arrive_expect_tx(&bars->full[stage], C::kTxBytes);
-        ptx::tma_load_2d_pair(sA + stage * A_STAGE, &tmA, &bars->full[stage], kb * BK, a_row);
-        ptx::tma_load_2d_pair(sB + stage * C::kBStage, &tmB, &bars->full[stage], kb * BK, b_row);
+        ptx::tma_load_2d_pair(sA + stage * A_STAGE, &tmA, &bars->full[stage], kb * KC::kStageK, a_row);
+        ptx::tma_load_2d_pair(sB + stage * C::kBStage, &tmB, &bars->full[stage], kb * KC::kStageK,
+                              b_row);
         last_stage = stage;
         last_phase = phase;
         if (++stage == C::kStages) {
@@ -275,7 +294,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int k = 0; k < BK / UMMA_K; ++k) {
           const uint64_t ad = ptx::smem_desc_k_sw128(a_addr + k * UMMA_K);
           const uint64_t bd = ptx::smem_desc_k_sw128(b_addr + k * UMMA_K);
-          ptx::mma_i8_pair(d_tmem, ad, bd, C::kIdesc, (kb | k) != 0 ? 1u : 0u);
+          if constexpr (kKind == kKindI8) {
+            ptx::mma_i8_pair(d_tmem, ad, bd, KC::kIdesc, (kb | k) != 0 ? 1u : 0u);
+          } else {
+            ptx::mma_f16_pair(d_tmem, ad, bd, KC::kIdesc, (kb | k) != 0 ? 1u : 0u);
+          }
         }
         issued = true;
         ptx::mma_commit_pair(&bars->empty[stage]);
@@ -310,8 +333,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::tc_fence_after();
       const int64_t m = static_cast<int64_t>(mb) * C::kTileM + rank * BM + row;
       const bool row_ok = m < p.M;
-      float scale = 0.f;
-      if (!p.out_s32 && row_ok) scale = p.s_tok[m] * (p.per_channel_scale ? 1.f : p.s_w[0]);
+      float scale = kKind == kKindI8 ? 0.f : 1.f;
+      if (kKind == kKindI8 && !p.out_s32 && row_ok) {
+        scale = p.s_tok[m] * (p.per_channel_scale ? 1.f : p.s_w[0]);
+      }
       const uint32_t t_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + acc * ACC_COLS;
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
@@ -321,12 +346,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int64_t n0 = static_cast<int64_t>(nb) * BN + c * 32;
         const int valid = n0 + 32 <= p.N ? 32 : (n0 + 16 <= p.N ? 16 : 0);
         if (row_ok && valid) {
-          if (p.out_s32) {
+          if (kKind == kKindI8 && p.out_s32) {
             store_s32_row32(static_cast<int32_t*>(p.out) + m * p.N + n0, r, valid);
           } else {
-            store_row32(static_cast<uint16_t*>(p.out) + m * p.N + n0, r, scale,
-                        p.per_channel_scale ? p.s_w + n0 : nullptr, p.bias ? p.bias + n0 : nullptr,
-                        valid, p.out_f16 != 0);
+            store_row32<kKind != kKindI8>(
+                static_cast<uint16_t*>(p.out) + m * p.N + n0, r, scale,
+                kKind == kKindI8 && p.per_channel_scale ? p.s_w + n0 : nullptr,
+                p.bias ? p.bias + n0 : nullptr, valid, p.out_f16 != 0);
           }
         }
       }
@@ -345,6 +371,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+__global__ void __launch_bounds__(kThreads, 1)
+    int8_gemm_tcgen05(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                      const Params p) {
+  gemm_pair<kKindI8>(tmA, tmB, p);
+}
+
+// x [M, K] and W [N, K] both bf16 (kF16 = false) or both fp16
+template <bool kF16>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm16_tcgen05(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const Params p) {
+  gemm_pair<kF16 ? kKindF16 : kKindBF16>(tmA, tmB, p);
+}
+
 // int8 [rows, K] row-major, box of `box_rows` x 128 bytes, 128-byte swizzle,
 // zero fill outside the tensor.
 bool encode_operand(CUtensorMap* map, const int8_t* base, int64_t rows, int64_t K, int box_rows) {
@@ -353,20 +393,31 @@ bool encode_operand(CUtensorMap* map, const int8_t* base, int64_t rows, int64_t 
                        static_cast<uint32_t>(box_rows));
 }
 
+// bf16 / fp16 [rows, K] row-major, box of `box_rows` x 64 elements (128 bytes),
+// 128-byte swizzle, zero fill outside the tensor.
+bool encode_operand16(CUtensorMap* map, const uint16_t* base, bool f16, int64_t rows, int64_t K,
+                      int box_rows) {
+  return encode_tma_2d(map, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                       base, static_cast<uint64_t>(K), static_cast<uint64_t>(rows),
+                       static_cast<uint64_t>(K) * 2, BK / 2, static_cast<uint32_t>(box_rows));
+}
+
 cudaError_t launch_pair(const GemmArgs& a, Params p, cudaStream_t stream) {
   using C = Cfg;
   CUtensorMap tmA, tmB;
-  if (!encode_operand(&tmA, a.A, a.M, a.K, BM) ||
-      !encode_operand(&tmB, a.B, a.N, a.K, C::kBRows)) {
-    return cudaErrorInvalidValue;
-  }
-  cudaError_t e = cudaFuncSetAttribute(int8_gemm_tcgen05,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+  const bool ok = a.ops16 ? encode_operand16(&tmA, a.A16, a.out_f16, a.M, a.K, BM) &&
+                                encode_operand16(&tmB, a.B16, a.out_f16, a.N, a.K, C::kBRows)
+                          : encode_operand(&tmA, a.A, a.M, a.K, BM) &&
+                                encode_operand(&tmB, a.B, a.N, a.K, C::kBRows);
+  if (!ok) return cudaErrorInvalidValue;
+  void (*kernel)(CUtensorMap, CUtensorMap, Params) =
+      !a.ops16 ? int8_gemm_tcgen05 : (a.out_f16 ? gemm16_tcgen05<true> : gemm16_tcgen05<false>);
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(C::kSmem));
   if (e != cudaSuccess) return e;
   p.m_tiles = static_cast<int>((a.M + C::kTileM - 1) / C::kTileM);
-  // all M-tiles per column sweep when A (M x K bytes) fits in half of L2
-  p.group_m = a.M * a.K <= (64ll << 20) ? p.m_tiles : 8;
+  // all M-tiles per column sweep when A (M x K elements) fits in half of L2
+  p.group_m = a.M * a.K * (a.ops16 ? 2 : 1) <= (64ll << 20) ? p.m_tiles : 8;
   const int tiles = p.m_tiles * p.n_tiles;
   const int per_unit = 2;  // CTAs per cluster
   const int max_units = sm_count() / per_unit;
@@ -385,7 +436,7 @@ cudaError_t launch_pair(const GemmArgs& a, Params p, cudaStream_t stream) {
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, int8_gemm_tcgen05, tmA, tmB, p);
+  return cudaLaunchKernelEx(&cfg, kernel, tmA, tmB, p);
 }
 
 }  // namespace
@@ -409,6 +460,25 @@ cudaError_t launch_int8_gemm(const GemmArgs& a, cudaStream_t stream) {
   // few tokens: the weight-streaming swap-AB kernel; otherwise CTA pairs
   // (256-row tiles) once there is more than one 128-row block of tokens
   if (a.M <= BM) return launch_int8_gemm_skinny(a, stream);
+  return launch_pair(a, p, stream);
+}
+
+cudaError_t launch_gemm16(const GemmArgs& a, cudaStream_t stream) {
+  if (a.M == 0) return cudaSuccess;
+  Params p;
+  cudaError_t se = status_word(&p.status);
+  if (se != cudaSuccess) return se;
+  p.s_tok = nullptr;
+  p.s_w = nullptr;
+  p.bias = a.bias;
+  p.out = a.out;
+  p.M = a.M;
+  p.N = a.N;
+  p.num_kb = static_cast<int>((2 * a.K + BK - 1) / BK);
+  p.n_tiles = static_cast<int>((a.N + BN - 1) / BN);
+  p.per_channel_scale = 0;
+  p.out_s32 = 0;
+  p.out_f16 = a.out_f16 ? 1 : 0;
   return launch_pair(a, p, stream);
 }
 

@@ -51,6 +51,10 @@ struct GemmArgs {
   int64_t M, N, K;
   bool out_s32;
   bool out_f16;          // y and bias are fp16 (else bf16)
+  // 16-bit operands (launch_gemm16): x [M, K] and W [N, K] in y's format
+  bool ops16 = false;
+  const uint16_t* A16 = nullptr;
+  const uint16_t* B16 = nullptr;
 };
 
 // Encodes the TMA descriptors and launches the tcgen05 GEMM.  Returns
@@ -59,6 +63,10 @@ cudaError_t launch_int8_gemm(const GemmArgs& a, cudaStream_t stream);
 
 // The few-token variant (M <= 128): swap-AB with the K split over a cluster.
 cudaError_t launch_int8_gemm_skinny(const GemmArgs& a, cudaStream_t stream);
+
+// y = f16(x W^T + bias) with 16-bit operands (a.ops16, a.A16, a.B16; bf16 or
+// fp16 as a.out_f16), fp32 accumulation on the same CTA-pair pipeline.
+cudaError_t launch_gemm16(const GemmArgs& a, cudaStream_t stream);
 
 // Enqueues the failure-detection self-test: a bounded wait that runs out
 // after `limit_ns` and records a timeout in the status word.

@@ -193,6 +193,16 @@ __host__ __device__ constexpr uint32_t idesc_i8(int M, int N) {
          | (static_cast<uint32_t>(M >> 4) << 24);   // M / 16
 }
 
+// Instruction descriptor of a kind::f16 MMA: fp32 accumulator, A and B both
+// bf16 (f16 = false) or both fp16, both K-major, M x N.
+__host__ __device__ constexpr uint32_t idesc_f16(int M, int N, bool f16) {
+  return (1u << 4)                                  // D format: F32
+         | ((f16 ? 0u : 1u) << 7)                   // A: F16 (0) or BF16 (1)
+         | ((f16 ? 0u : 1u) << 10)                  // B: same type as A
+         | (static_cast<uint32_t>(N >> 3) << 17)    // N / 8
+         | (static_cast<uint32_t>(M >> 4) << 24);   // M / 16
+}
+
 // ---------------------------------------------------------------- CTA pairs
 // A cluster of two CTAs on two SMs shares one tcgen05 MMA (cta_group::2).  In
 // the cluster's shared window bit 24 of a shared address selects the CTA of
@@ -251,6 +261,18 @@ __device__ __forceinline__ void mma_i8_pair(uint32_t d_tmem, uint64_t a_desc, ui
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::2.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// The same for 16-bit operands (kind::f16: K = 16 elements = 32 bytes per
+// instruction, fp32 accumulator).
+__device__ __forceinline__ void mma_f16_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                             uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }

@@ -62,6 +62,8 @@ typedef struct convrot_rotation_s* convrot_rotation_t;  /* opaque, owned by the 
 /* Workspace queries (convrot_workspace_bytes). */
 #define CONVROT_OP_LINEAR_INT8 1         /* all M tokens in one pass */
 #define CONVROT_OP_LINEAR_INT8_SLICED 2  /* slices of at most 2N tokens (see convrot_linear_int8) */
+#define CONVROT_OP_LINEAR_DEQUANT 3      /* the decoded weight of convrot_linear_dequant */
+#define CONVROT_OP_LINEAR_CHECKED 4      /* convrot_linear_checked, its first call included */
 
 /* Library version, major * 10000 + minor * 100 + patch. */
 int convrot_version(void);
@@ -196,6 +198,82 @@ convrot_status convrot_linear_int8_noalloc(const convrot_bf16* x, int64_t M, int
 size_t convrot_noalloc_scratch_bytes(void);
 
 /*
+ * The default path's matmul (Invoke docs "int8 Compute", opening section:
+ * without int8 compute a layer unpacks its weight to BF16 or FP16 and
+ * multiplies in that precision):
+ *   y[m, n] = bf16_rn( sum_k x[m, k] * W[n, k] + bias[n] )
+ * x [M, K] bf16, W [N, K] bf16 (typically W_hat of convrot_dequant_derotate),
+ * bias [N] bf16 or NULL -> y [M, N] bf16.  The products are exact in fp32 and
+ * are summed in fp32 on the tensor cores in an order of the kernel's choosing;
+ * the bias is added in fp32 before the one rounding.  Limits: N % 16 == 0,
+ * K % 16 == 0, K <= 131072, 16-byte aligned pointers; M == 0 is a no-op.
+ */
+convrot_status convrot_dense_linear(const convrot_bf16* x, int64_t M, int64_t K, int64_t N,
+                                    const convrot_bf16* W, const convrot_bf16* bias,
+                                    convrot_bf16* y, convrot_stream_t stream);
+
+/*
+ * The default path of a ConvRot int8 layer (Invoke docs "int8 Compute": a
+ * layer that does not run in int8 dequantizes its weight on every forward):
+ * convrot_dequant_derotate into the workspace, then convrot_dense_linear.
+ * Arguments as convrot_linear_int8.  `ws` (256-byte aligned) holds the decoded
+ * weight: convrot_workspace_bytes(CONVROT_OP_LINEAR_DEQUANT, M, N, K) =
+ * 2*N*K rounded up to 256 bytes, else CONVROT_ERR_WORKSPACE.
+ */
+convrot_status convrot_linear_dequant(const convrot_bf16* x, int64_t M, int64_t K, int64_t N,
+                                      convrot_rotation_t R, const int8_t* Wq, const float* s_w,
+                                      int64_t s_w_len, const convrot_bf16* bias, convrot_bf16* y,
+                                      void* ws, size_t ws_bytes, convrot_stream_t stream);
+
+/*
+ * The int8-compute forward with the first-call check against the default path
+ * (Invoke docs "int8 Compute", "When something goes wrong" and "Memory"):
+ *   - Calls are grouped by key: (device, N, K, G, 16-bit format, M bucket),
+ *     with M bucket = ceil(log2(M)) (1 token: bucket 0).
+ *   - The first call of a key runs convrot_linear_int8 into y, then the default
+ *     path (convrot_linear_dequant) for the first R = min(M, CONVROT_CHECK_ROWS)
+ *     rows, and compares the two on those R rows.  They match when no kernel
+ *     reported a timeout, every y value is finite where the default path's is,
+ *     and cosine(y, y_default) >= the threshold (convrot_check_min_cosine; the
+ *     pages give none, the default is 0.99).  This call synchronizes `stream`.
+ *   - On a mismatch, or when an int8-path launch fails, the call prints one
+ *     warning to stderr, latches the device onto the default path for the rest
+ *     of the process and overwrites y with the default path's result for all
+ *     M rows.
+ *   - Later calls of a checked key, on a device that is not latched, are
+ *     convrot_linear_int8 (asynchronous); on a latched device every call is
+ *     convrot_linear_dequant.
+ *   - `path` (HOST pointer, may be NULL) receives CONVROT_PATH_INT8 or
+ *     CONVROT_PATH_DEQUANT: the path whose result y holds.
+ *   - `ws` (256-byte aligned): convrot_workspace_bytes(CONVROT_OP_LINEAR_CHECKED,
+ *     M, N, K) bytes, the larger of the int8 forward's and the check's needs
+ *     (the decoded weight, R rows of output and a few sums).
+ * Argument errors are those of convrot_linear_int8 and latch nothing.
+ */
+#define CONVROT_CHECK_ROWS 256
+#define CONVROT_PATH_INT8 1
+#define CONVROT_PATH_DEQUANT 2
+convrot_status convrot_linear_checked(const convrot_bf16* x, int64_t M, int64_t K, int64_t N,
+                                      convrot_rotation_t R, const int8_t* Wq, const float* s_w,
+                                      int64_t s_w_len, const convrot_bf16* bias, convrot_bf16* y,
+                                      void* ws, size_t ws_bytes, int* path,
+                                      convrot_stream_t stream);
+
+/*
+ * State of the check (host side, thread-safe).  convrot_check_state reports
+ * for CUDA device `device` whether it is latched onto the default path (1/0)
+ * and how many keys have been checked on it.  convrot_check_reset forgets
+ * every checked key and latch on every device (as a restart would).
+ * convrot_check_set_min_cosine sets the match threshold (0 < t <= 1.5; a value
+ * above 1 makes every check fail, which lets a caller exercise the fallback
+ * without a faulty kernel); convrot_check_min_cosine returns it.
+ */
+convrot_status convrot_check_state(int device, int* latched, int* checked_keys);
+void convrot_check_reset(void);
+convrot_status convrot_check_set_min_cosine(double threshold);
+double convrot_check_min_cosine(void);
+
+/*
  * fp16 forms.  The pages' int8 layers run with BF16 or FP16 activations and
  * refuse only FP32 (Invoke docs "int8 Compute": the opening section unpacks
  * each layer "to BF16 or FP16", and the table of layers that keep
@@ -224,6 +302,18 @@ convrot_status convrot_linear_int8_f16(const convrot_f16* x, int64_t M, int64_t 
                                        convrot_rotation_t R, const int8_t* Wq, const float* s_w,
                                        int64_t s_w_len, const convrot_f16* bias, convrot_f16* y,
                                        void* ws, size_t ws_bytes, convrot_stream_t stream);
+convrot_status convrot_dense_linear_f16(const convrot_f16* x, int64_t M, int64_t K, int64_t N,
+                                        const convrot_f16* W, const convrot_f16* bias,
+                                        convrot_f16* y, convrot_stream_t stream);
+convrot_status convrot_linear_dequant_f16(const convrot_f16* x, int64_t M, int64_t K, int64_t N,
+                                          convrot_rotation_t R, const int8_t* Wq, const float* s_w,
+                                          int64_t s_w_len, const convrot_f16* bias, convrot_f16* y,
+                                          void* ws, size_t ws_bytes, convrot_stream_t stream);
+convrot_status convrot_linear_checked_f16(const convrot_f16* x, int64_t M, int64_t K, int64_t N,
+                                          convrot_rotation_t R, const int8_t* Wq, const float* s_w,
+                                          int64_t s_w_len, const convrot_f16* bias, convrot_f16* y,
+                                          void* ws, size_t ws_bytes, int* path,
+                                          convrot_stream_t stream);
 
 /* Bytes of workspace an operation needs (0 if none); 0 for an unknown op. */
 size_t convrot_workspace_bytes(int op, int64_t M, int64_t N, int64_t K);

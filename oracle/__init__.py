@@ -17,6 +17,7 @@ from .convrot_oracle import (  # noqa: F401
     f16_round,
     int8_gemm_acc,
     linear_dense,
+    linear_dequant,
     linear_int8,
     quantize_symmetric,
     quantize_weight,

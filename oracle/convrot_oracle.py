@@ -230,6 +230,20 @@ def linear_int8(x, Wq, s_w, R, bias=None, fmt: str = "bf16"):
     return epilogue(acc, s_tok, s_w, bias, fmt), xq, s_tok, acc
 
 
+def linear_dequant(x, Wq, s_w, R, bias=None, fmt: str = "bf16") -> np.ndarray:
+    """The default path of a ConvRot layer: decode the weight to the 16-bit
+    format, then y = f16(x . W_hat^T + b), the exact sum rounded once.
+
+    [INT8C] opening section (a layer that does not compute in int8 unpacks its
+    weight to BF16 or FP16 and multiplies in that precision) and "When
+    something goes wrong" (the default path is what the first int8 result is
+    checked against).  The sum is taken in float64; the pages fix no
+    summation precision for the matmul.  Returns float64 [M, N].
+    """
+    W_hat = dequant_derotate(Wq, s_w, R, fmt)
+    return round16(linear_dense(x, W_hat, bias), fmt)
+
+
 def linear_dense(x, W, bias=None) -> np.ndarray:
     """Unquantized reference layer y = x . W^T + b in float64 (no rounding)."""
     y = as_f64(x) @ as_f64(W).T

@@ -105,6 +105,47 @@ def test_workspace_size():
     assert sliced == lib.convrot_workspace_bytes(cr.OP_LINEAR_INT8, 2048, 1024, K)
 
 
+def test_default_path_and_checked_workspace_sizes():
+    M, N, K = 4608, 11520, 3840
+    dq = lib.convrot_workspace_bytes(cr.OP_LINEAR_DEQUANT, M, N, K)
+    assert dq == 2 * N * K  # already a multiple of 256
+    chk = lib.convrot_workspace_bytes(cr.OP_LINEAR_CHECKED, M, N, K)
+    # the decoded weight + 256 rows of output + the sums, or the int8 codes if larger
+    assert chk == max(dq + 2 * 256 * N + 256, lib.convrot_workspace_bytes(cr.OP_LINEAR_INT8, M, N, K))
+    # few tokens: only M rows are checked
+    assert lib.convrot_workspace_bytes(cr.OP_LINEAR_CHECKED, 3, 1024, 1024) == (
+        2 * 1024 * 1024 + 256 * ((2 * 3 * 1024 + 255) // 256) + 256)
+
+
+def test_check_state_on_the_host():
+    cr.check_reset()
+    assert cr.check_state(0) == (False, 0)
+    assert cr.check_min_cosine() == 0.99
+    cr.check_set_min_cosine(1.2)
+    assert cr.check_min_cosine() == 1.2
+    for bad in (0.0, -1.0, 1.6, float("nan")):
+        with pytest.raises(cr.ConvRotError) as e:
+            cr.check_set_min_cosine(bad)
+        assert e.value.status == cr.INVALID_ARG
+    cr.check_set_min_cosine(0.99)
+    assert lib.convrot_check_state(-1, None, None) == cr.INVALID_ARG
+
+
+def test_checked_rejects_before_device():
+    f = lib.convrot_linear_checked
+    path = ctypes.c_int(7)
+    # no rotation handle, then no workspace: errors before any CUDA call, nothing latched
+    assert f(FAKE, 8, 256, 32, None, FAKE, FAKE, 1, None, FAKE, FAKE, 1 << 24, ctypes.byref(path),
+             None) == cr.INVALID_ARG
+    assert path.value == 0
+    g = lib.convrot_linear_dequant
+    assert g(FAKE, 8, 256, 24, None, FAKE, FAKE, 1, None, FAKE, FAKE, 1 << 24, None) == cr.INVALID_ARG
+    assert g(FAKE, 8, 256, 32, None, FAKE, FAKE, 1, None, FAKE, None, 0, None) == cr.WORKSPACE
+    assert lib.convrot_dense_linear(FAKE, 8, 64, 24, FAKE, None, FAKE, None) == cr.INVALID_ARG
+    assert lib.convrot_dense_linear(MISALIGNED, 8, 64, 32, FAKE, None, FAKE, None) == cr.ALIGNMENT
+    assert cr.check_state(0) == (False, 0)
+
+
 def test_linear_rejects_before_device():
     f = lib.convrot_linear_int8
     assert f(FAKE, 8, 256, 24, None, FAKE, FAKE, 1, None, FAKE, FAKE, 1 << 20, None) == cr.INVALID_ARG

@@ -265,12 +265,40 @@ def check_f16_round(o):
                                   [[51.5, 48.5, 51.5, 48.5]])
 
 
+def check_default_path(o):
+    """The default path (decode, then one rounding of x . W_hat^T + b) against
+    exact rational arithmetic on a small layer whose sums are exact in float64,
+    and the unit-vector closed form y[0, n] = f16(W_hat[n, k] + b[n])."""
+    from fractions import Fraction
+    rng = np.random.default_rng(11)
+    M, N, K = 3, 5, 8
+    Wq = rng.integers(-127, 128, (N, K), dtype=np.int64).astype(np.int8)
+    s_w = np.float32(0.1)  # not a power of two: the decoded weight must be rounded
+    x = o.bf16_round(rng.standard_normal((M, K)))
+    b = o.bf16_round(rng.standard_normal(N))
+    for fmt in ("bf16", "f16"):
+        W_hat = o.dequant_derotate(Wq, s_w, H4_HALF, fmt)
+        y = o.linear_dequant(x, Wq, s_w, H4_HALF, b, fmt)
+        for m in range(M):
+            for n in range(N):
+                exact = sum(Fraction(float(x[m, k])) * Fraction(float(W_hat[n, k])) for k in range(K))
+                exact += Fraction(float(b[n]))
+                assert float(exact) == exact  # representable: one rounding below
+                assert y[m, n] == o.round16(float(exact), fmt)
+        e = np.zeros((1, K))
+        e[0, 2] = 1.0
+        np.testing.assert_array_equal(o.linear_dequant(e, Wq, s_w, H4_HALF, b, fmt)[0],
+                                      o.round16(W_hat[:, 2] + b, fmt))
+        np.testing.assert_array_equal(o.linear_dequant(0 * e, Wq, s_w, H4_HALF, b, fmt)[0],
+                                      o.round16(b, fmt))
+
+
 CHECKS = [
     check_f16_round, check_worked_example, check_block_rotate_bruteforce, check_block_rotate_direction,
     check_rotation_identity, check_round_trip, check_bf16_round, check_quantize_symmetric,
     check_act_quant_properties, check_zero_token, check_gemm_bruteforce, check_gemm_extremes,
     check_epilogue_closed_forms, check_weight_decode_accuracy, check_layer_accuracy,
-    check_rotation_helps_outliers,
+    check_rotation_helps_outliers, check_default_path,
 ]
 
 
@@ -363,6 +391,12 @@ def _bug_f16_no_subnormals(v):
     return np.where(np.abs(r) > 65504.0, np.copysign(np.inf, v), r)
 
 
+def _bug_default_path_unrounded_weight(x, Wq, s_w, R, bias=None, fmt="bf16"):
+    W = np.float64(np.float32(s_w)) * real_oracle.block_rotate(np.asarray(Wq, np.float64),
+                                                               real_oracle.as_f64(R).T)
+    return real_oracle.round16(real_oracle.linear_dense(x, W, bias), fmt)
+
+
 def _bug_scale_255(W, R):
     W_rot = real_oracle.block_rotate(W, R)
     s_w = np.float32(np.max(np.abs(W_rot)) / 255)
@@ -380,6 +414,7 @@ MUTANTS = {
     "weight_scale_255": dict(quantize_weight=_bug_scale_255),
     "f16_ten_significant_bits": dict(f16_round=_bug_f16_ten_bits),
     "f16_without_subnormals": dict(f16_round=_bug_f16_no_subnormals),
+    "default_path_unrounded_weight": dict(linear_dequant=_bug_default_path_unrounded_weight),
 }
 
 
