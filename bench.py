@@ -42,8 +42,8 @@ INT8_PER_BF16 = 2.0  # nominal dense int8 : bf16 tensor throughput (4.5 : 2.25 P
 # DRAM bytes per launch from ncu (dram__bytes_read.sum + dram__bytes_write.sum),
 # averaged over the three GEMM launches of one Z-Image step, valid only for the
 # kernel source they were taken on (first 16 hex digits of its sha256).
-NCU_TRAFFIC = {"int8_gemm_tcgen05": (120.19e6 + 101.99e6 + 151.16e6) / 3}
-NCU_TRAFFIC_SOURCE_SHA = {"int8_gemm_tcgen05": "b5f9eeca52952e70"}
+NCU_TRAFFIC = {"int8_gemm_tcgen05": (120.24e6 + 102.27e6 + 151.76e6) / 3}
+NCU_TRAFFIC_SOURCE_SHA = {"int8_gemm_tcgen05": "401d1e52793f0ba8"}
 
 
 def source_sha(rel: str) -> str:
@@ -578,6 +578,69 @@ def run_sweep(args):
     return 0
 
 
+def run_default_path(args):
+    """int8 compute against the pages' default path on the workload's linears
+    (Invoke docs "int8 Compute": the default path decodes the weight and
+    multiplies in 16 bits on every forward).  Per linear, CUDA events around one
+    call on L2-flushed inputs: convrot_linear_int8 (rotate+quantize, int8 GEMM),
+    convrot_linear_dequant (decode, 16-bit GEMM) and the 16-bit GEMM alone on a
+    decoded weight; one JSON line."""
+    import torch
+
+    import activation_quantized_linear_b200 as cr
+    torch.cuda.set_device(0)
+    hbm_gbs, bf16_tflops, _, peak_kind = load_peaks()
+    act = torch.float16 if args.dtype == "f16" else torch.bfloat16
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    flush_rd = torch.ones(64 << 20, dtype=torch.float32, device="cuda")
+
+    def timed(fn, n):
+        ts = []
+        for k in range(n + 3):
+            flush.fill_(k & 0xFF)
+            flush_rd.sum()
+            torch.cuda._sleep(400_000)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            if k >= 3:
+                ts.append(e0.elapsed_time(e1))
+        return statistics.median(ts)
+
+    rows = []
+    for i, lin in enumerate(workloads.WORKLOADS[args.workload]):
+        inp = workloads.make_layer_inputs(lin, i, dtype=act)
+        M, N, K = lin.M, lin.N, lin.K
+        rot = cr.Rotation(inp.R)
+        Wq, s_w = cr.quantize_weight(inp.W.cuda(), rot)
+        x, b = inp.x.cuda(), inp.bias.cuda()
+        y = torch.empty((M, N), dtype=act, device="cuda")
+        ws_i8 = torch.empty(cr.workspace_bytes(M, N, K), dtype=torch.uint8, device="cuda")
+        ws_dq = torch.empty(cr.workspace_bytes(M, N, K, op=cr.OP_LINEAR_DEQUANT),
+                            dtype=torch.uint8, device="cuda")
+        W_hat = cr.dequant_derotate(Wq, s_w, rot, dtype=act)
+        t_i8 = timed(lambda: cr.linear_int8(x, Wq, s_w, rot, b, out=y, workspace=ws_i8), args.steps)
+        t_dq = timed(lambda: cr.linear_dequant(x, Wq, s_w, rot, b, out=y, workspace=ws_dq),
+                     args.steps)
+        t_dense = timed(lambda: cr.dense_linear(x, W_hat, b, out=y), args.steps)
+        flops = 2.0 * M * N * K
+        rows.append({"linear": f"{lin.name}:M{M}xK{K}->N{N}", "int8_ms": t_i8, "dequant_ms": t_dq,
+                     "dense16_ms": t_dense, "int8_speedup_over_default": t_dq / t_i8,
+                     "dense16_tflops": flops / t_dense / 1e9,
+                     "dense16_frac_bf16_peak": flops / t_dense / 1e9 / bf16_tflops})
+        del Wq, W_hat, ws_i8, ws_dq, y
+    total_i8 = sum(r["int8_ms"] for r in rows)
+    total_dq = sum(r["dequant_ms"] for r in rows)
+    print(json.dumps({"compare": "int8_compute_vs_default_path", "workload": args.workload,
+                      "dtype": args.dtype, "linears": rows,
+                      "int8_speedup_over_default": total_dq / total_i8,
+                      "bf16_peak_tflops": bf16_tflops, "peak": peak_kind,
+                      "timing": "median of --steps single calls, CUDA events, L2 flushed before each"}))
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -591,6 +654,8 @@ def main():
     ap.add_argument("--ref-rows", type=int, default=64)
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--default-path", action="store_true",
+                    help="time int8 compute against the default path (decode + 16-bit GEMM) instead")
     ap.add_argument("--sweep", action="store_true",
                     help="time the group-size / skinny-M sweep and the decode sweep instead")
     args = ap.parse_args()
@@ -598,6 +663,8 @@ def main():
         raise SystemExit("--warmup must be >= 3")
     if args.sweep:
         return run_sweep(args)
+    if args.default_path:
+        return run_default_path(args)
     lins = workloads.WORKLOADS[args.workload]
     if args.impl == "reference":
         return run_reference(args, lins)
