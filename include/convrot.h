@@ -235,7 +235,10 @@ convrot_status convrot_linear_dequant(const convrot_bf16* x, int64_t M, int64_t 
  *     rows, and compares the two on those R rows.  They match when no kernel
  *     reported a timeout, every y value is finite where the default path's is,
  *     and cosine(y, y_default) >= the threshold (convrot_check_min_cosine; the
- *     pages give none, the default is 0.99).  This call synchronizes `stream`.
+ *     pages give none, the default is 0.99).  This call synchronizes `stream`
+ *     and reads the device status word (convrot_check_status), so make it
+ *     outside CUDA stream capture; it attributes any timeout recorded since
+ *     the last status check to the int8 kernels.
  *   - On a mismatch, or when an int8-path launch fails, the call prints one
  *     warning to stderr, latches the device onto the default path for the rest
  *     of the process and overwrites y with the default path's result for all

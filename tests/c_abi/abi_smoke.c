@@ -41,6 +41,24 @@ int main(void) {
                                (const float*)fake, 1, NULL, 0, 32, 64, (convrot_f16*)fake,
                                NULL) == CONVROT_OK); /* M = 0: nothing to do */
   EXPECT(convrot_selftest_wait_timeout(0, NULL) == CONVROT_ERR_INVALID_ARG);
+
+  /* the default path and the checked forward */
+  EXPECT(convrot_workspace_bytes(CONVROT_OP_LINEAR_DEQUANT, 64, 1024, 512) == 2u * 1024u * 512u);
+  EXPECT(convrot_workspace_bytes(CONVROT_OP_LINEAR_CHECKED, 4608, 1024, 512) >=
+         convrot_workspace_bytes(CONVROT_OP_LINEAR_DEQUANT, 4608, 1024, 512) +
+             2u * CONVROT_CHECK_ROWS * 1024u);
+  EXPECT(convrot_dense_linear((const convrot_bf16*)fake, 8, 64, 24, (const convrot_bf16*)fake, NULL,
+                              (convrot_bf16*)fake, NULL) == CONVROT_ERR_INVALID_ARG);
+  int path = -1, latched = -1, keys = -1;
+  EXPECT(convrot_linear_checked((const convrot_bf16*)fake, 8, 256, 32, NULL, (const int8_t*)fake,
+                                (const float*)fake, 1, NULL, (convrot_bf16*)fake, fake, 1u << 24,
+                                &path, NULL) == CONVROT_ERR_INVALID_ARG);
+  EXPECT(path == 0);
+  EXPECT(convrot_check_state(0, &latched, &keys) == CONVROT_OK && latched == 0 && keys == 0);
+  EXPECT(convrot_check_set_min_cosine(2.0) == CONVROT_ERR_INVALID_ARG);
+  EXPECT(convrot_check_min_cosine() == 0.99);
+  EXPECT(CONVROT_PATH_INT8 != CONVROT_PATH_DEQUANT);
+  convrot_check_reset();
   printf("c abi ok\n");
   return 0;
 }
