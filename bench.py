@@ -419,6 +419,9 @@ def run_ours(args, lins):
     if rank != 0:
         return 0
     tops_frac = gemm_tops / int8_peak
+    # the tensor cores' own int8 rate on this GPU (after the timed region):
+    # context for the denominator, which stays the measured bf16 rate x 2
+    issue_tops = cr.measure_int8_mma_rate(32768)
     out = {
         "metric": "int8 ConvRot linear TOPS (rotate+quant+GEMM)",
         "value": value, "unit": "TOPS", "n_gpus": world, "steps": args.steps,
@@ -430,6 +433,8 @@ def run_ours(args, lins):
             "peak": int8_peak, "unit": "TFLOP/s", "frac": tops_frac, "traffic": traffic,
             "peak_source": f"{peak_src} bf16 {bf16_tflops} TFLOP/s (burst) x {INT8_PER_BF16} "
                            f"nominal int8:bf16",
+            "int8_issue_loop_tops": issue_tops,
+            "frac_of_issue_loop": gemm_tops / issue_tops if issue_tops > 0 else None,
         },
         "kernels": {
             "rotate_quant_act": {"ms": rqa_mean.tolist(), "GB/s": rqa_gbs,
@@ -625,18 +630,32 @@ def run_default_path(args):
         t_dq = timed(lambda: cr.linear_dequant(x, Wq, s_w, rot, b, out=y, workspace=ws_dq),
                      args.steps)
         t_dense = timed(lambda: cr.dense_linear(x, W_hat, b, out=y), args.steps)
+        # a library int8 GEMM for reference: torch._int_mm (int32 out, no epilogue)
+        try:
+            xq, _ = cr.rotate_quant_act(x, rot)
+            Wt = Wq.t()  # [K, N] view of the [N, K] codes
+            torch._int_mm(xq, Wt)
+            t_intmm = timed(lambda: torch._int_mm(xq, Wt), args.steps)
+            t_ours = timed(lambda: cr.int8_gemm_s32(xq, Wq), args.steps)
+            intmm = {"torch_int_mm_ms": t_intmm, "torch_int_mm_tops": 2.0 * M * N * K / t_intmm / 1e9,
+                     "int8_gemm_s32_ms": t_ours, "int8_gemm_s32_tops": 2.0 * M * N * K / t_ours / 1e9}
+            del xq
+        except Exception as exc:  # noqa: BLE001 (a reference point only)
+            intmm = {"torch_int_mm": f"unavailable: {type(exc).__name__}: {exc}"[:200]}
         flops = 2.0 * M * N * K
         rows.append({"linear": f"{lin.name}:M{M}xK{K}->N{N}", "int8_ms": t_i8, "dequant_ms": t_dq,
                      "dense16_ms": t_dense, "int8_speedup_over_default": t_dq / t_i8,
                      "dense16_tflops": flops / t_dense / 1e9,
-                     "dense16_frac_bf16_peak": flops / t_dense / 1e9 / bf16_tflops})
+                     "dense16_frac_bf16_peak": flops / t_dense / 1e9 / bf16_tflops, **intmm})
         del Wq, W_hat, ws_i8, ws_dq, y
+    issue_tops = cr.measure_int8_mma_rate(32768)
     total_i8 = sum(r["int8_ms"] for r in rows)
     total_dq = sum(r["dequant_ms"] for r in rows)
     print(json.dumps({"compare": "int8_compute_vs_default_path", "workload": args.workload,
                       "dtype": args.dtype, "linears": rows,
                       "int8_speedup_over_default": total_dq / total_i8,
                       "bf16_peak_tflops": bf16_tflops, "peak": peak_kind,
+                      "int8_issue_loop_tops": issue_tops,
                       "timing": "median of --steps single calls, CUDA events, L2 flushed before each"}))
     return 0
 

@@ -340,6 +340,19 @@ convrot_status convrot_check_status(convrot_stream_t stream);
  */
 convrot_status convrot_selftest_wait_timeout(int limit_ms, convrot_stream_t stream);
 
+/*
+ * Measured int8 tensor-core rate of the current device, in TOP/s (no
+ * counterpart on the pages: a cross-check for the int8 GEMM's roofline
+ * denominator).  Every SM issues `iters` x 4 back-to-back
+ * tcgen05.mma.kind::i8 of 128 x 256 x 32 on operands of pseudo-random bytes
+ * held in shared memory, with nothing loaded or stored; one launch is timed
+ * with CUDA events.
+ * iters in [1, 200000] (32768 runs for about 10 ms), else
+ * CONVROT_ERR_INVALID_ARG.  Synchronizes `stream`; `tops` is a HOST pointer.
+ * Returns CONVROT_ERR_TIMEOUT if the kernel's bounded wait ran out.
+ */
+convrot_status convrot_measure_int8_mma_rate(int iters, double* tops, convrot_stream_t stream);
+
 /* Message of the last failure on the calling thread ("" if none). */
 const char* convrot_last_error_string(void);
 

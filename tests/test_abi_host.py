@@ -146,6 +146,14 @@ def test_checked_rejects_before_device():
     assert cr.check_state(0) == (False, 0)
 
 
+def test_mma_rate_rejects_before_device():
+    tops = ctypes.c_double(0.0)
+    f = lib.convrot_measure_int8_mma_rate
+    assert f(0, ctypes.byref(tops), None) == cr.INVALID_ARG
+    assert f(200001, ctypes.byref(tops), None) == cr.INVALID_ARG
+    assert f(100, None, None) == cr.INVALID_ARG
+
+
 def test_linear_rejects_before_device():
     f = lib.convrot_linear_int8
     assert f(FAKE, 8, 256, 24, None, FAKE, FAKE, 1, None, FAKE, FAKE, 1 << 20, None) == cr.INVALID_ARG
