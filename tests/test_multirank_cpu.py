@@ -68,3 +68,23 @@ def test_world_size_must_match_gpus(monkeypatch):
     monkeypatch.setenv("WORLD_SIZE", "4")
     with pytest.raises(SystemExit):
         bench.dist_setup(2)
+
+
+def test_issue_loop_measurement_failure_keeps_the_bench_line():
+    """The tensor-core rate is context for the roofline: if measuring it fails,
+    the bench reports None instead of losing its JSON line."""
+    import bench
+
+    class Failing:
+        @staticmethod
+        def measure_int8_mma_rate(iters):
+            raise RuntimeError("no device")
+
+    class Working:
+        @staticmethod
+        def measure_int8_mma_rate(iters):
+            assert iters == 32768
+            return 4321.0
+
+    assert bench.issue_loop_tops(Failing) is None
+    assert bench.issue_loop_tops(Working) == 4321.0
