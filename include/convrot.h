@@ -26,7 +26,9 @@
  *     owns only the device copy of R inside a rotation handle.  No entry point
  *     allocates device memory, except convrot_rotation_create.
  *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL means the
- *     legacy default stream).  Argument errors return at once, before any
+ *     legacy default stream), except three that synchronize it and say so:
+ *     convrot_check_status, the first call of a key in
+ *     convrot_linear_checked, and convrot_measure_int8_mma_rate.  Argument errors return at once, before any
  *     launch, and leave the outputs untouched.  A launch failure returns
  *     CONVROT_ERR_CUDA.  A wait inside a kernel that runs out of time (about a
  *     second) makes that kernel stop and record CONVROT_ERR_TIMEOUT in a device
