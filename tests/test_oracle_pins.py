@@ -194,6 +194,11 @@ def check_epilogue_closed_forms(o):
     np.testing.assert_array_equal(o.epilogue(acc, np.float32([1.0]), np.float32(1.0)), [[0, 1, -3, 2.0 ** 20]])
     # 257 is not a bf16 (needs 9 bits) and is half way between 256 and 258 -> 256 (even)
     np.testing.assert_array_equal(o.epilogue(np.array([[257]]), np.float32([1.0]), np.float32(1.0)), [[256.0]])
+    # one rounding of acc*s + bias: 1027 * 2^-10 = 1 + 0.375 ulp, plus 2^-9 = 0.25 ulp
+    # gives 1 + 0.625 ulp -> 1 + 2^-7; rounding the product first would give 1
+    np.testing.assert_array_equal(
+        o.epilogue(np.array([[1027]]), np.float32([2.0 ** -10]), np.float32(1.0), np.array([2.0 ** -9])),
+        [[1.0 + 2.0 ** -7]])
 
 
 def check_weight_decode_accuracy(o):
@@ -397,6 +402,30 @@ def _bug_default_path_unrounded_weight(x, Wq, s_w, R, bias=None, fmt="bf16"):
     return real_oracle.round16(real_oracle.linear_dense(x, W, bias), fmt)
 
 
+def _bug_act_absmax_before_rotation(x, R):
+    x_rot = real_oracle.block_rotate(x, R)
+    s_tok = (np.max(np.abs(real_oracle.as_f64(x)), axis=1) / 127).astype(np.float32)
+    return real_oracle.quantize_symmetric(x_rot, s_tok[:, None]), s_tok
+
+
+def _bug_weight_scale_per_row(W, R):
+    W_rot = real_oracle.block_rotate(W, R)
+    s = (np.max(np.abs(W_rot), axis=1) / 127).astype(np.float32)
+    return real_oracle.quantize_symmetric(W_rot, s[:, None]), np.float32(np.max(s))
+
+
+def _bug_epilogue_rounds_before_bias(acc, s_tok, s_w, bias=None, fmt="bf16"):
+    y = real_oracle.epilogue(acc, s_tok, s_w, None, fmt)
+    if bias is not None:
+        y = y + real_oracle.as_f64(bias)[None, :]
+    return real_oracle.round16(y, fmt)
+
+
+def _bug_decode_with_R(Wq, s_w, R, fmt="bf16"):
+    return real_oracle.round16(np.float64(np.float32(s_w)) * real_oracle.block_rotate(
+        np.asarray(Wq, np.float64), real_oracle.as_f64(R)), fmt)
+
+
 def _bug_scale_255(W, R):
     W_rot = real_oracle.block_rotate(W, R)
     s_w = np.float32(np.max(np.abs(W_rot)) / 255)
@@ -415,6 +444,10 @@ MUTANTS = {
     "f16_ten_significant_bits": dict(f16_round=_bug_f16_ten_bits),
     "f16_without_subnormals": dict(f16_round=_bug_f16_no_subnormals),
     "default_path_unrounded_weight": dict(linear_dequant=_bug_default_path_unrounded_weight),
+    "act_absmax_before_rotation": dict(rotate_quant_act=_bug_act_absmax_before_rotation),
+    "weight_scale_per_row": dict(quantize_weight=_bug_weight_scale_per_row),
+    "epilogue_rounds_before_bias": dict(epilogue=_bug_epilogue_rounds_before_bias),
+    "decode_multiplies_by_R_not_RT": dict(dequant_derotate=_bug_decode_with_R),
 }
 
 
