@@ -426,6 +426,32 @@ def _bug_decode_with_R(Wq, s_w, R, fmt="bf16"):
         np.asarray(Wq, np.float64), real_oracle.as_f64(R)), fmt)
 
 
+def _bug_codes_reach_minus_128(v, scale):
+    v32 = np.asarray(v, np.float64).astype(np.float32)
+    s32 = np.broadcast_to(np.asarray(scale, np.float32), v32.shape)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        q = np.rint(v32 / s32)
+    return np.clip(np.where(s32 == 0, 0, q), -128, 127).astype(np.int8)
+
+
+def _bug_groups_strided(A, R):
+    # K split into G strided groups instead of K/G contiguous blocks of G
+    A = real_oracle.as_f64(A)
+    R = real_oracle.as_f64(R)
+    G = R.shape[0]
+    rows, K = A.shape
+    B = A.reshape(rows, G, K // G).transpose(0, 2, 1)
+    return (B @ R).transpose(0, 2, 1).reshape(rows, K)
+
+
+def _bug_f16_ties_away(v):
+    v = np.asarray(v, np.float64)
+    _, e = np.frexp(v)
+    ulp = np.ldexp(1.0, np.maximum(e, -13) - 11)
+    r = np.sign(v) * np.floor(np.abs(v) / ulp + 0.5) * ulp
+    return np.where(np.abs(r) > 65504.0, np.copysign(np.inf, v), r)
+
+
 def _bug_scale_255(W, R):
     W_rot = real_oracle.block_rotate(W, R)
     s_w = np.float32(np.max(np.abs(W_rot)) / 255)
@@ -448,6 +474,9 @@ MUTANTS = {
     "weight_scale_per_row": dict(quantize_weight=_bug_weight_scale_per_row),
     "epilogue_rounds_before_bias": dict(epilogue=_bug_epilogue_rounds_before_bias),
     "decode_multiplies_by_R_not_RT": dict(dequant_derotate=_bug_decode_with_R),
+    "codes_reach_minus_128": dict(quantize_symmetric=_bug_codes_reach_minus_128),
+    "groups_strided_over_K": dict(block_rotate=_bug_groups_strided),
+    "f16_ties_away_from_zero": dict(f16_round=_bug_f16_ties_away),
 }
 
 
