@@ -62,6 +62,11 @@ def _check_linear(cr, lin, index, R, name):
     assert xq.min() >= -127 and xq.max() <= 127
     amax = np.abs(xq.astype(np.int32)).max(axis=1)
     assert np.all((amax == 127) | (s_tok == 0)), name
+    # every token's codes and scale against the oracle (full tensors)
+    xq_all, s_all = oracle.rotate_quant_act(inp.x, R)
+    np.testing.assert_allclose(s_tok, s_all, rtol=1e-6)
+    assert_codes_close(xq, xq_all)
+    del xq_all, s_all
     # sampled rows against the oracle
     rows = sample_rows(lin.M, 256, seed=index)
     x_s = inp.x[rows]
