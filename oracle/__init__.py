@@ -24,4 +24,5 @@ from .convrot_oracle import (  # noqa: F401
     rel_l2,
     rotate_quant_act,
     round16,
+    weight_scale_column,
 )

@@ -30,6 +30,15 @@ Readings where the pages leave a step open (each is a choice, stated once):
   Quantization Works", `--scaling_mode tensor`) and one per token for the
   activation ([INT8C], opening section), both absmax / 127, symmetric codes
   in [-127, 127] (never -128).
+* per-output-channel weight scale: a weight may instead carry one float32
+  scale per output channel, s_w[n] = max_k |W_rot[n, k]| / 127 ([PR194]
+  "Summary", Z-Image's fused QKV, whose per-output-channel scale splits with
+  its weight; "QA Instructions", int8 carries one scale per output channel).
+  It multiplies along the OUTPUT axis: row n of the decoded weight and column
+  n of the layer output.  [PR194]'s scale-layout fix names the mistake this
+  excludes: a length-N scale left to trailing-axis broadcasting scales the
+  input axis (wrong values for square weights, a size error for the rest).
+  A scale array of any length other than 1 or N is refused.
 * rounding: round half to even, no learned/SVD rounding ([CTQ] `--simple`).
 * the code decision round(v / s) is taken in float32, the CUDA kernels'
   precision, since the pages fix none: v and s are first rounded to float32,
@@ -144,30 +153,54 @@ def quantize_symmetric(v, scale) -> np.ndarray:
 # the layer's operations
 # ---------------------------------------------------------------------------
 
-def quantize_weight(W, R):
+def weight_scale_column(s_w, N) -> np.ndarray:
+    """The weight scale laid along the output axis, as float64 [N, 1]: a scalar
+    (or a length-1 array) is one scale per tensor, a length-N array one scale
+    per output channel (row n of the weight).  Any other length is refused,
+    not broadcast.
+
+    [PR194] "Summary" (per-output-channel scales split with their weight) and
+    its scale-layout fix (a `[out]` scale must not scale the input axis).
+    """
+    s = np.asarray(s_w, dtype=np.float32).reshape(-1)
+    if s.size == 1:
+        return np.full((N, 1), np.float64(s[0]))
+    if s.size != N:
+        raise ValueError(f"weight scale of length {s.size} for {N} output channels")
+    return s.astype(np.float64)[:, None]
+
+
+def quantize_weight(W, R, per_channel: bool = False):
     """Offline weight quantization: rotate W in G-blocks along its input
-    dimension, take one per-tensor scale absmax / 127, round to int8.
+    dimension, take the scale absmax / 127 over the whole tensor (or, with
+    per_channel, over each output channel's row), round to int8.
 
     [CTQ] "How INT8 ConvRot Quantization Works": `--int8 --scaling_mode tensor
-    --simple --convrot --convrot-group-size G` ("one global scale per tensor").
-    Returns (Wq int8 [N, K], s_w float32 scalar).
+    --simple --convrot --convrot-group-size G` ("one global scale per tensor");
+    [PR194] "Summary" and "QA Instructions" for the per-output-channel form.
+    Returns (Wq int8 [N, K], s_w float32 scalar, or float32 [N] per channel).
     """
     W_rot = block_rotate(W, R)
+    if per_channel:
+        a = np.max(np.abs(W_rot), axis=1) if W_rot.shape[1] else np.zeros(W_rot.shape[0])
+        s_w = (a / INT8_QMAX).astype(np.float32)
+        return quantize_symmetric(W_rot, s_w[:, None]), s_w
     a = np.max(np.abs(W_rot)) if W_rot.size else 0.0
     s_w = np.float32(a / INT8_QMAX)
     return quantize_symmetric(W_rot, s_w), s_w
 
 
 def dequant_derotate(Wq, s_w, R, fmt: str = "bf16") -> np.ndarray:
-    """Default (weight-decode) path: W_hat = bf16(s_w * Wq . B_R^T) (fp16 with
-    fmt="f16").
+    """Default (weight-decode) path: W_hat[n] = bf16(s_w[n] * Wq[n] . B_R^T)
+    (fp16 with fmt="f16"); s_w is one scale per tensor or per output channel.
 
     [PR194] "Summary": each quantized layer "dequantizes and derotates per
     forward"; the derotation is the product [out, in/G, G] @ [G, G].
     Returns the 16-bit values as float64 [N, K].
     """
     R = as_f64(R)
-    return round16(np.float64(np.float32(s_w)) * block_rotate(np.asarray(Wq, np.float64), R.T), fmt)
+    Wq = np.asarray(Wq, np.float64)
+    return round16(weight_scale_column(s_w, Wq.shape[0]) * block_rotate(Wq, R.T), fmt)
 
 
 def rotate_quant_act(x, R):
@@ -205,16 +238,17 @@ def int8_gemm_acc(xq, Wq) -> np.ndarray:
 
 
 def epilogue(acc, s_tok, s_w, bias=None, fmt: str = "bf16") -> np.ndarray:
-    """int8_compute, step 3: y = bf16(acc * s_tok[m] * s_w + bias[n]) (fp16 with
-    fmt="f16").
+    """int8_compute, step 3: y = bf16(acc * s_tok[m] * s_w[n] + bias[n]) (fp16
+    with fmt="f16"); s_w is one scale per tensor or per output channel n.
 
     [INT8C] opening section and "Layer / Why" table (outputs are BF16/FP16);
     the bias is the nn.Linear bias the layer replaces ([PR194] "Summary").
     Returns the 16-bit values as float64 [M, N].
     """
-    y = (np.asarray(acc, np.float64)
+    acc = np.asarray(acc, np.float64)
+    y = (acc
          * np.asarray(s_tok, np.float32).astype(np.float64)[:, None]
-         * np.float64(np.float32(s_w)))
+         * weight_scale_column(s_w, acc.shape[1]).T)
     if bias is not None:
         y = y + as_f64(bias)[None, :]
     return round16(y, fmt)

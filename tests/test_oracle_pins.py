@@ -298,7 +298,80 @@ def check_default_path(o):
                                       o.round16(b, fmt))
 
 
+def _fraction_array(strs):
+    from fractions import Fraction
+    return np.array([float(Fraction(v)) for v in strs])
+
+
+def check_per_channel_worked_example(o):
+    """Hand-derived per-output-channel example
+    (tests/golden/per_channel_worked_example.json): a non-square layer end to
+    end, a square decode whose input-axis reading differs, and an epilogue
+    with M != N."""
+    g = _golden("per_channel_worked_example.json")
+    x, W, b = (np.array(g[k], np.float64) for k in ("A_x", "A_W", "A_bias"))
+    Wq, s_w = o.quantize_weight(W, H4_HALF, per_channel=True)
+    np.testing.assert_array_equal(Wq, np.array(g["A_Wq"]))
+    np.testing.assert_array_equal(s_w, _fraction_array(g["A_s_w_exact"]).astype(np.float32))
+    np.testing.assert_array_equal(o.dequant_derotate(Wq, s_w, H4_HALF), np.array(g["A_W_hat"]))
+    y, xq, s_tok, acc = o.linear_int8(x, Wq, s_w, H4_HALF, b)
+    np.testing.assert_array_equal(acc, np.array(g["A_acc"]))
+    np.testing.assert_array_equal(y, np.array(g["A_y"]))
+    np.testing.assert_array_equal(o.linear_dense(x, W, b), np.array(g["A_y_dense"]))
+    np.testing.assert_array_equal(
+        o.epilogue(np.array(g["C_acc"], np.int32), np.array(g["C_s_tok"], np.float32),
+                   np.array(g["C_s_w"], np.float32), np.array(g["C_bias"])),
+        np.array(g["C_y"]))
+
+
+def check_per_channel_square_decode(o):
+    """Part B of the per-channel golden: a square weight, where the input-axis
+    broadcast of PR #194's scale-layout fix raises no size error and only the
+    values can show the wrong axis."""
+    g = _golden("per_channel_worked_example.json")
+    np.testing.assert_array_equal(
+        o.dequant_derotate(np.array(g["B_Wq"], np.int8), np.array(g["B_s_w"], np.float32), H4_HALF),
+        np.array(g["B_W_hat"]))
+
+
+def check_per_channel_properties(o):
+    """Per output channel: s_w[n] = max_k |W_rot[n, k]| / 127 (float32), every
+    row's largest code is +-127, |W_rot - q s_w| <= s_w / 2; a constant scale
+    vector decodes and rescales exactly like the per-tensor scalar; a scale of
+    any length other than 1 or N is refused rather than broadcast."""
+    lin = workloads.Linear("t", 5, 256, 48, G=64)
+    inp = workloads.make_layer_inputs(lin, 3)
+    R = workloads.sylvester_rotation(64)
+    Wq, s_w = o.quantize_weight(inp.W, R, per_channel=True)
+    W_rot = o.block_rotate(inp.W, R)
+    assert s_w.shape == (48,) and s_w.dtype == np.float32
+    np.testing.assert_array_equal(s_w, (np.max(np.abs(W_rot), axis=1) / 127).astype(np.float32))
+    np.testing.assert_array_equal(np.max(np.abs(Wq.astype(np.int32)), axis=1), 127)
+    err = np.abs(W_rot - Wq.astype(np.float64) * s_w[:, None].astype(np.float64))
+    assert np.all(err <= s_w[:, None] * (0.5 + 1e-5))
+    c = np.float32(1.7e-3)
+    np.testing.assert_array_equal(o.dequant_derotate(Wq, np.full(48, c), R), o.dequant_derotate(Wq, c, R))
+    acc = np.random.default_rng(8).integers(-2 ** 20, 2 ** 20, (3, 48)).astype(np.int32)
+    s_tok = np.array([1e-2, 2e-3, 0.0], np.float32)
+    np.testing.assert_array_equal(o.epilogue(acc, s_tok, np.full(48, c)), o.epilogue(acc, s_tok, c))
+    # column n of the output scales with s_w[n] alone (a power of two: exact)
+    s_vec = np.ones(48, np.float32)
+    s_vec[7] = 4.0
+    y1 = o.epilogue(acc, s_tok, s_vec)
+    y0 = o.epilogue(acc, s_tok, np.float32(1.0))
+    np.testing.assert_array_equal(y1[:, 7], 4.0 * y0[:, 7])
+    np.testing.assert_array_equal(np.delete(y1, 7, axis=1), np.delete(y0, 7, axis=1))
+    for bad in (np.ones(47, np.float32), np.ones(3, np.float32)):
+        for call in (lambda: o.dequant_derotate(Wq, bad, R), lambda: o.epilogue(acc, s_tok, bad)):
+            try:
+                call()
+            except ValueError:
+                continue
+            raise AssertionError("a weight scale of the wrong length was accepted")
+
+
 CHECKS = [
+    check_per_channel_worked_example, check_per_channel_square_decode, check_per_channel_properties,
     check_f16_round, check_worked_example, check_block_rotate_bruteforce, check_block_rotate_direction,
     check_rotation_identity, check_round_trip, check_bf16_round, check_quantize_symmetric,
     check_act_quant_properties, check_zero_token, check_gemm_bruteforce, check_gemm_extremes,
@@ -408,7 +481,9 @@ def _bug_act_absmax_before_rotation(x, R):
     return real_oracle.quantize_symmetric(x_rot, s_tok[:, None]), s_tok
 
 
-def _bug_weight_scale_per_row(W, R):
+def _bug_weight_scale_per_row(W, R, per_channel=False):
+    if per_channel:
+        return real_oracle.quantize_weight(W, R, True)
     W_rot = real_oracle.block_rotate(W, R)
     s = (np.max(np.abs(W_rot), axis=1) / 127).astype(np.float32)
     return real_oracle.quantize_symmetric(W_rot, s[:, None]), np.float32(np.max(s))
@@ -452,13 +527,49 @@ def _bug_f16_ties_away(v):
     return np.where(np.abs(r) > 65504.0, np.copysign(np.inf, v), r)
 
 
-def _bug_scale_255(W, R):
+def _bug_scale_255(W, R, per_channel=False):
+    if per_channel:
+        return real_oracle.quantize_weight(W, R, True)
     W_rot = real_oracle.block_rotate(W, R)
     s_w = np.float32(np.max(np.abs(W_rot)) / 255)
     return real_oracle.quantize_symmetric(W_rot, s_w), s_w
 
 
+def _bug_decode_scale_on_input_axis(Wq, s_w, R, fmt="bf16"):
+    # PR #194's broadcast trap: a [N] scale aligned with the trailing (input) axis
+    s = np.asarray(s_w, np.float32).astype(np.float64)
+    return real_oracle.round16(
+        real_oracle.block_rotate(np.asarray(Wq, np.float64), real_oracle.as_f64(R).T) * s, fmt)
+
+
+def _bug_epilogue_scale_on_token_axis(acc, s_tok, s_w, bias=None, fmt="bf16"):
+    acc = np.asarray(acc, np.float64)
+    s = np.asarray(s_w, np.float32).astype(np.float64).reshape(-1)
+    y = acc * np.asarray(s_tok, np.float32).astype(np.float64)[:, None] * (s[:, None] if s.size > 1 else s)
+    if bias is not None:
+        y = y + real_oracle.as_f64(bias)[None, :]
+    return real_oracle.round16(y, fmt)
+
+
+def _bug_channel_scales_collapsed(s_w, N):
+    # a per-channel vector silently reduced to its first entry
+    s = np.asarray(s_w, np.float32).reshape(-1)
+    return np.full((N, 1), np.float64(s[0]))
+
+
+def _bug_per_channel_codes_with_tensor_scale(W, R, per_channel=False):
+    Wq, s = real_oracle.quantize_weight(W, R, False)
+    if not per_channel:
+        return Wq, s
+    W_rot = real_oracle.block_rotate(W, R)
+    return Wq, (np.max(np.abs(W_rot), axis=1) / 127).astype(np.float32)
+
+
 MUTANTS = {
+    "decode_scale_on_input_axis": dict(dequant_derotate=_bug_decode_scale_on_input_axis),
+    "epilogue_scale_on_token_axis": dict(epilogue=_bug_epilogue_scale_on_token_axis),
+    "channel_scales_collapsed": dict(weight_scale_column=_bug_channel_scales_collapsed),
+    "per_channel_codes_with_tensor_scale": dict(quantize_weight=_bug_per_channel_codes_with_tensor_scale),
     "skip_derotation": dict(dequant_derotate=_bug_skip_derotation),
     "transposed_rotation": dict(block_rotate=_bug_transposed_rotation),
     "drop_bias": dict(epilogue=_bug_drop_bias),
@@ -490,3 +601,11 @@ def test_planted_mistake_is_caught(name):
         except (AssertionError, ValueError, OverflowError):
             failed.append(check.__name__)
     assert failed, f"planted mistake {name!r} passed every check"
+
+
+def test_input_axis_scale_fails_on_square_values():
+    """The input-axis mistake raises a size error on a non-square weight; on the
+    square weight it must still fail, on the values alone."""
+    m = _mutant(**MUTANTS["decode_scale_on_input_axis"])
+    with pytest.raises(AssertionError):
+        check_per_channel_square_decode(m)
