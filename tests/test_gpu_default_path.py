@@ -160,11 +160,10 @@ def test_linear_dequant_per_channel_scale():
     rng = np.random.default_rng(5)
     s = (float(s_w.item()) * (1 + 0.2 * rng.random(640))).astype(np.float32)
     y = cr.linear_dequant(inp.x.cuda(), Wq, torch.from_numpy(s).cuda(), rot, inp.bias.cuda())
-    W_hat = oracle.round16(s.astype(np.float64)[:, None]
-                           * oracle.block_rotate(Wq.cpu().numpy().astype(np.float64),
-                                                 oracle.as_f64(inp.R).T), "bf16")
+    Wq_h = Wq.cpu().numpy()
+    W_hat = oracle.dequant_derotate(Wq_h, s, inp.R)
     x64, b64 = oracle.as_f64(inp.x), oracle.as_f64(inp.bias)
-    ref = oracle.round16(oracle.linear_dense(x64, W_hat, b64), "bf16")
+    ref = oracle.linear_dequant(x64, Wq_h, s, inp.R, b64)
     got = oracle.as_f64(y.cpu())
     assert np.all(np.abs(got - ref) <= bf16_ulp(ref) + dense_bound(x64, W_hat, b64, 512))
 

@@ -131,8 +131,7 @@ def test_dequant_derotate_f16_scales(G):
     s[::3] = 2.0 ** -12
     W_hat = cr.dequant_derotate(torch.from_numpy(Wq).cuda(), torch.from_numpy(s).cuda(), rot,
                                 dtype=F16)
-    ref = oracle.f16_round(s.astype(np.float64)[:, None]
-                           * oracle.block_rotate(Wq.astype(np.float64), R.astype(np.float64).T))
+    ref = oracle.dequant_derotate(Wq, s, R, "f16")
     np.testing.assert_array_equal(f16_bits(W_hat), oracle.f16_bits(ref))
 
 
@@ -156,10 +155,7 @@ def test_int8_gemm_f16(M, N, K, with_bias, per_channel):
     out.check()
     acc = oracle.int8_gemm_acc(a, b)
     sw = np.broadcast_to(np.atleast_1d(s_w).astype(np.float64), (N,))
-    y64 = acc.astype(np.float64) * s_tok.astype(np.float64)[:, None] * sw[None, :]
-    if bias is not None:
-        y64 = y64 + oracle.as_f64(bias)[None, :]
-    ref = oracle.f16_round(y64)
+    ref = oracle.epilogue(acc, s_tok, s_w, bias, "f16")
     got = oracle.as_f64(y.cpu())
     mag = np.abs(acc.astype(np.float64) * s_tok.astype(np.float64)[:, None] * sw[None, :])
     if bias is not None:
