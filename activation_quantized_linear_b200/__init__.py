@@ -142,6 +142,55 @@ def _need(t: torch.Tensor, name: str, dtype: torch.dtype, ndim: int) -> None:
 FLOAT16 = (torch.bfloat16, torch.float16)
 
 
+def _tensor(t, name: str) -> None:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+
+
+def _shape(t: torch.Tensor | None, name: str, shape: tuple) -> None:
+    """An optional caller-supplied tensor must have exactly `shape`."""
+    if t is None:
+        return
+    _tensor(t, name)
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _layer_shapes(x, Wq, s_w, bias, out) -> tuple[int, int, int]:
+    """The layer's size contract, checked before anything reaches the C ABI
+    (which takes raw pointers and cannot see a size): Wq [N, K] for x [M, K],
+    one weight scale or N of them (s_w None: no scale), N biases, out [M, N].
+    Returns (M, K, N)."""
+    for t, name in ((x, "x"), (Wq, "Wq")):
+        _tensor(t, name)
+    if x.dim() != 2 or Wq.dim() != 2:
+        raise ValueError(f"x and Wq must be 2-D, got {tuple(x.shape)} and {tuple(Wq.shape)}")
+    M, K = x.shape
+    N = Wq.shape[0]
+    if Wq.shape[1] != K:
+        raise ValueError(f"Wq has {Wq.shape[1]} input features, x has {K}")
+    if s_w is not None:
+        _tensor(s_w, "s_w")
+        if s_w.numel() not in (1, N):
+            raise ValueError(f"s_w must hold 1 or N = {N} scales, got {s_w.numel()}")
+    if bias is not None:
+        _tensor(bias, "bias")
+        if bias.numel() != N:
+            raise ValueError(f"bias must hold N = {N} values, got {bias.numel()}")
+    _shape(out, "out", (M, N))
+    return M, K, N
+
+
+def _on_current_device(**tensors) -> None:
+    """Every tensor handed to the library must live on the current CUDA device:
+    the library launches there and resolves its per-device state (rotation
+    copy, static scratch, status word) there."""
+    dev = torch.cuda.current_device()
+    for name, t in tensors.items():
+        if t is not None and (t.device.type != "cuda" or t.device.index != dev):
+            raise ValueError(f"{name} is on {t.device}; the current device is cuda:{dev}")
+
+
 def _need16(t: torch.Tensor, name: str, ndim: int) -> None:
     """A bf16 or fp16 tensor (the layer's two activation formats)."""
     if not isinstance(t, torch.Tensor):
@@ -207,10 +256,17 @@ class Rotation:
 def quantize_weight(W: torch.Tensor, rot: Rotation, Wq: torch.Tensor | None = None,
                     s_w: torch.Tensor | None = None):
     """W [N, K] bf16 or fp16 -> (Wq [N, K] int8, s_w [1] float32)."""
+    _tensor(W, "W")
+    if W.dim() == 2:
+        _shape(Wq, "Wq", tuple(W.shape))
+        _shape(s_w, "s_w", (1,))
     _need16(W, "W", 2)
     N, K = W.shape
     Wq = torch.empty((N, K), dtype=torch.int8, device=W.device) if Wq is None else Wq
     s_w = torch.empty(1, dtype=torch.float32, device=W.device) if s_w is None else s_w
+    _need(Wq, "Wq", torch.int8, 2)
+    _need(s_w, "s_w", torch.float32, 1)
+    _on_current_device(W=W, Wq=Wq, s_w=s_w)
     _check(_fn("convrot_quantize_weight", W.dtype)(_ptr(W), N, K, rot.handle, _ptr(Wq), _ptr(s_w),
                                                     _stream()))
     return Wq, s_w
@@ -221,11 +277,18 @@ def dequant_derotate(Wq: torch.Tensor, s_w: torch.Tensor, rot: Rotation,
                      dtype: torch.dtype = torch.bfloat16) -> torch.Tensor:
     """Wq [N, K] int8, s_w [1] or [N] float32 -> W_hat [N, K] in `dtype` (bf16 or
     fp16; the dtype of `out` when given)."""
+    _tensor(Wq, "Wq")
+    _tensor(s_w, "s_w")
+    if Wq.dim() == 2:
+        if s_w.numel() not in (1, Wq.shape[0]):
+            raise ValueError(f"s_w must hold 1 or N = {Wq.shape[0]} scales, got {s_w.numel()}")
+        _shape(out, "out", tuple(Wq.shape))
     _need(Wq, "Wq", torch.int8, 2)
     _need(s_w, "s_w", torch.float32, 1)
     N, K = Wq.shape
     out = torch.empty((N, K), dtype=dtype, device=Wq.device) if out is None else out
     _need16(out, "out", 2)
+    _on_current_device(Wq=Wq, s_w=s_w, out=out)
     _check(_fn("convrot_dequant_derotate", out.dtype)(_ptr(Wq), _ptr(s_w), s_w.numel(), N, K,
                                                        rot.handle, _ptr(out), _stream()))
     return out
@@ -234,10 +297,17 @@ def dequant_derotate(Wq: torch.Tensor, s_w: torch.Tensor, rot: Rotation,
 def rotate_quant_act(x: torch.Tensor, rot: Rotation, xq: torch.Tensor | None = None,
                      s_tok: torch.Tensor | None = None):
     """x [M, K] bf16 or fp16 -> (xq [M, K] int8, s_tok [M] float32)."""
+    _tensor(x, "x")
+    if x.dim() == 2:
+        _shape(xq, "xq", tuple(x.shape))
+        _shape(s_tok, "s_tok", (x.shape[0],))
     _need16(x, "x", 2)
     M, K = x.shape
     xq = torch.empty((M, K), dtype=torch.int8, device=x.device) if xq is None else xq
     s_tok = torch.empty(M, dtype=torch.float32, device=x.device) if s_tok is None else s_tok
+    _need(xq, "xq", torch.int8, 2)
+    _need(s_tok, "s_tok", torch.float32, 1)
+    _on_current_device(x=x, xq=xq, s_tok=s_tok)
     _check(_fn("convrot_rotate_quant_act", x.dtype)(_ptr(x), M, K, rot.handle, _ptr(xq),
                                                      _ptr(s_tok), _stream()))
     return xq, s_tok
@@ -249,20 +319,21 @@ def int8_gemm(xq: torch.Tensor, s_tok: torch.Tensor, Wq: torch.Tensor, s_w: torc
     """y = xq . Wq^T * s_tok[:, None] * s_w + bias, rounded once to a 16-bit
     float: the dtype of `out` when given, else `dtype`, else the bias's dtype,
     else bf16.  The bias, if any, is in the output's dtype."""
+    M, K, N = _layer_shapes(xq, Wq, s_w, bias, out)
+    _tensor(s_tok, "s_tok")
+    if s_tok.numel() != M:
+        raise ValueError(f"s_tok must hold M = {M} scales, got {s_tok.numel()}")
     _need(xq, "xq", torch.int8, 2)
     _need(Wq, "Wq", torch.int8, 2)
     _need(s_tok, "s_tok", torch.float32, 1)
     _need(s_w, "s_w", torch.float32, 1)
-    M, K = xq.shape
-    N = Wq.shape[0]
-    if Wq.shape[1] != K:
-        raise ValueError("xq and Wq disagree on K")
     if out is None:
         dtype = dtype or (bias.dtype if bias is not None else torch.bfloat16)
         out = torch.empty((M, N), dtype=dtype, device=xq.device)
     _need16(out, "out", 2)
     if bias is not None:
         _need(bias, "bias", out.dtype, 1)
+    _on_current_device(xq=xq, s_tok=s_tok, Wq=Wq, s_w=s_w, bias=bias, out=out)
     _check(_fn("convrot_int8_gemm", out.dtype)(_ptr(xq), _ptr(s_tok), _ptr(Wq), _ptr(s_w),
                                                 s_w.numel(), _ptr(bias), M, N, K, _ptr(out),
                                                 _stream()))
@@ -271,13 +342,19 @@ def int8_gemm(xq: torch.Tensor, s_tok: torch.Tensor, Wq: torch.Tensor, s_w: torc
 
 def int8_gemm_s32(xq: torch.Tensor, Wq: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
     """acc = xq . Wq^T as int32 (diagnostic form of the GEMM)."""
+    _tensor(xq, "xq")
+    _tensor(Wq, "Wq")
+    if xq.dim() == 2 and Wq.dim() == 2:
+        if Wq.shape[1] != xq.shape[1]:
+            raise ValueError(f"Wq has {Wq.shape[1]} input features, xq has {xq.shape[1]}")
+        _shape(out, "out", (xq.shape[0], Wq.shape[0]))
     _need(xq, "xq", torch.int8, 2)
     _need(Wq, "Wq", torch.int8, 2)
     M, K = xq.shape
     N = Wq.shape[0]
-    if Wq.shape[1] != K:
-        raise ValueError("xq and Wq disagree on K")
     out = torch.empty((M, N), dtype=torch.int32, device=xq.device) if out is None else out
+    _need(out, "out", torch.int32, 2)
+    _on_current_device(xq=xq, Wq=Wq, out=out)
     _check(_lib.convrot_int8_gemm_s32(_ptr(xq), _ptr(Wq), M, N, K, _ptr(out), _stream()))
     return out
 
@@ -295,6 +372,7 @@ def _workspace(workspace: torch.Tensor | None, need: int, device) -> torch.Tenso
     if workspace is None:
         return torch.empty(max(need, 1), dtype=torch.uint8, device=device)
     _need(workspace, "workspace", torch.uint8, 1)
+    _on_current_device(workspace=workspace)
     return workspace
 
 
@@ -303,18 +381,19 @@ def linear_int8(x: torch.Tensor, Wq: torch.Tensor, s_w: torch.Tensor, rot: Rotat
                 workspace: torch.Tensor | None = None) -> torch.Tensor:
     """The int8-compute forward: rotate+quantize x per token, int8 GEMM, rescale.
     x, bias and the output share one 16-bit float format (bf16 or fp16)."""
+    M, K, N = _layer_shapes(x, Wq, s_w, bias, out)
     _need16(x, "x", 2)
     _need(Wq, "Wq", torch.int8, 2)
     _need(s_w, "s_w", torch.float32, 1)
     if bias is not None:
         _need(bias, "bias", x.dtype, 1)
-    M, K = x.shape
-    N = Wq.shape[0]
     need = workspace_bytes(M, N, K)
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=x.device)
+    _need(workspace, "workspace", torch.uint8, 1)
     out = torch.empty((M, N), dtype=x.dtype, device=x.device) if out is None else out
     _need(out, "out", x.dtype, 2)
+    _on_current_device(x=x, Wq=Wq, s_w=s_w, bias=bias, out=out, workspace=workspace)
     _check(_fn("convrot_linear_int8", x.dtype)(_ptr(x), M, K, N, rot.handle, _ptr(Wq), _ptr(s_w),
                                                 s_w.numel(), _ptr(bias), _ptr(out),
                                                 _ptr(workspace), workspace.numel(), _stream()))
@@ -327,14 +406,15 @@ def linear_int8_noalloc(x: torch.Tensor, Wq: torch.Tensor, s_w: torch.Tensor, ro
     """linear_int8 for callers that cannot allocate device memory: the
     intermediate codes and scales live in the library's static scratch
     (noalloc_scratch_bytes() bytes per GPU).  Pass `out` to allocate nothing."""
+    M, K, N = _layer_shapes(x, Wq, s_w, bias, out)
     _need(x, "x", torch.bfloat16, 2)
     _need(Wq, "Wq", torch.int8, 2)
     _need(s_w, "s_w", torch.float32, 1)
     if bias is not None:
         _need(bias, "bias", torch.bfloat16, 1)
-    M, K = x.shape
-    N = Wq.shape[0]
     out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device) if out is None else out
+    _need(out, "out", torch.bfloat16, 2)
+    _on_current_device(x=x, Wq=Wq, s_w=s_w, bias=bias, out=out)
     _check(_lib.convrot_linear_int8_noalloc(_ptr(x), M, K, N, rot.handle, _ptr(Wq), _ptr(s_w),
                                             s_w.numel(), _ptr(bias), _ptr(out), _stream()))
     return out
@@ -344,31 +424,30 @@ def dense_linear(x: torch.Tensor, W: torch.Tensor, bias: torch.Tensor | None = N
                  out: torch.Tensor | None = None) -> torch.Tensor:
     """The default path's matmul: y = x W^T + bias, x, W, bias and y in one
     16-bit float format, fp32 accumulation on the tensor cores."""
+    _tensor(W, "W")
+    M, K, N = _layer_shapes(x, W, None, bias, out)
     _need16(x, "x", 2)
     _need(W, "W", x.dtype, 2)
     if bias is not None:
         _need(bias, "bias", x.dtype, 1)
-    M, K = x.shape
-    N = W.shape[0]
-    if W.shape[1] != K:
-        raise ValueError(f"W has {W.shape[1]} input features, x has {K}")
     out = torch.empty((M, N), dtype=x.dtype, device=x.device) if out is None else out
     _need(out, "out", x.dtype, 2)
+    _on_current_device(x=x, W=W, bias=bias, out=out)
     _check(_fn("convrot_dense_linear", x.dtype)(_ptr(x), M, K, N, _ptr(W), _ptr(bias), _ptr(out),
                                                  _stream()))
     return out
 
 
 def _linear_args(x, Wq, s_w, bias, out):
+    M, K, N = _layer_shapes(x, Wq, s_w, bias, out)
     _need16(x, "x", 2)
     _need(Wq, "Wq", torch.int8, 2)
     _need(s_w, "s_w", torch.float32, 1)
     if bias is not None:
         _need(bias, "bias", x.dtype, 1)
-    M, K = x.shape
-    N = Wq.shape[0]
     out = torch.empty((M, N), dtype=x.dtype, device=x.device) if out is None else out
     _need(out, "out", x.dtype, 2)
+    _on_current_device(x=x, Wq=Wq, s_w=s_w, bias=bias, out=out)
     return M, K, N, out
 
 
