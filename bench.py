@@ -40,10 +40,10 @@ FALLBACK_BF16_TFLOPS = 1590.0
 INT8_PER_BF16 = 2.0  # nominal dense int8 : bf16 tensor throughput (4.5 : 2.25 POPS)
 
 # DRAM bytes per launch from ncu (dram__bytes_read.sum + dram__bytes_write.sum),
-# averaged over the three GEMM launches of one Z-Image step, valid only for the
+# averaged over the GEMM launches of one step of a workload, valid only for the
 # kernel source they were taken on (first 16 hex digits of its sha256).
-NCU_TRAFFIC = {"int8_gemm_tcgen05": (120.24e6 + 102.27e6 + 151.76e6) / 3}
-NCU_TRAFFIC_SOURCE_SHA = {"int8_gemm_tcgen05": "401d1e52793f0ba8"}
+NCU_TRAFFIC = {("int8_gemm_tcgen05", "zimage_dit_block"): (120.24e6 + 102.27e6 + 151.76e6) / 3}
+NCU_TRAFFIC_SOURCE_SHA = {("int8_gemm_tcgen05", "zimage_dit_block"): "401d1e52793f0ba8"}
 
 
 def source_sha(rel: str) -> str:
@@ -366,7 +366,7 @@ def run_ours(args, lins):
 
     gemm_src = "activation_quantized_linear_b200/csrc/int8_gemm.cu"
     traffic = None
-    key = "int8_gemm_tcgen05"
+    key = ("int8_gemm_tcgen05", args.workload)
     if NCU_TRAFFIC.get(key) and NCU_TRAFFIC_SOURCE_SHA.get(key) == source_sha(gemm_src):
         traffic = NCU_TRAFFIC[key]
 
@@ -677,7 +677,7 @@ def main():
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="zimage_dit_block",
+    ap.add_argument("--workload", default="wan22_a14b_video_dit",
                     choices=[k for k in workloads.WORKLOADS if k != "group_size_sweep"])
     ap.add_argument("--dtype", default="bf16", choices=["bf16", "f16"],
                     help="16-bit float format of activations, bias, outputs and the decoded weight")
