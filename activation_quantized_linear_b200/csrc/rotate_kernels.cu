@@ -93,11 +93,13 @@ __device__ __forceinline__ uint64_t mulrz2(uint64_t a, uint64_t b) {
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
-__device__ __forceinline__ void sts128(uint32_t addr, uint64_t a, uint64_t b) {
-  asm volatile("st.shared.v2.b64 [%0], {%1, %2};" ::"r"(addr), "l"(a), "l"(b) : "memory");
+__device__ __forceinline__ void sts64(uint32_t addr, uint64_t a) {
+  asm volatile("st.shared.b64 [%0], %1;" ::"r"(addr), "l"(a) : "memory");
 }
-__device__ __forceinline__ void lds128(uint32_t addr, uint64_t& a, uint64_t& b) {
-  asm volatile("ld.shared.v2.b64 {%0, %1}, [%2];" : "=l"(a), "=l"(b) : "r"(addr) : "memory");
+__device__ __forceinline__ uint64_t lds64(uint32_t addr) {
+  uint64_t a;
+  asm volatile("ld.shared.b64 %0, [%1];" : "=l"(a) : "r"(addr) : "memory");
+  return a;
 }
 
 // ---------------------------------------------------------------- loads
@@ -136,6 +138,39 @@ __device__ __forceinline__ void widen16_32(const uint4 (&u)[4], uint64_t (&P)[kP
   }
 }
 
+// 16-bit words -> P[i] = (p[2i] + p[2i + 1], p[2i] - p[2i + 1]): the widening
+// and butterfly bit 0 together.  The high element is widened to float32; the
+// low one enters the sm_100 mixed-precision add and subtract as a 16-bit
+// operand, which is converted exactly, so each result is the float32 sum
+// rounded once, as in fwht32's own bit-0 stage.
+template <bool kF16>
+__device__ __forceinline__ void widen_stage0_32(const uint4 (&u)[4], uint64_t (&P)[kPairs]) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t w[4] = {u[j].x, u[j].y, u[j].z, u[j].w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      float sum, dif;
+      if constexpr (kF16) {
+        asm("{\n\t.reg .b16 lo, hi;\n\t.reg .f32 h;\n\tmov.b32 {lo, hi}, %2;\n\t"
+            "cvt.f32.f16 h, hi;\n\t"
+            "add.rn.f32.f16 %0, lo, h;\n\t"
+            "sub.rn.f32.f16 %1, lo, h;\n\t}"
+            : "=f"(sum), "=f"(dif)
+            : "r"(w[k]));
+      } else {
+        const float h = __uint_as_float(w[k] & 0xffff0000u);
+        asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+            "add.rn.f32.bf16 %0, lo, %3;\n\t"
+            "sub.rn.f32.bf16 %1, lo, %3;\n\t}"
+            : "=f"(sum), "=f"(dif)
+            : "r"(w[k]), "f"(h));
+      }
+      P[4 * j + k] = pk(sum, dif);
+    }
+  }
+}
+
 // raw int8 words -> P[i] = (p[2i], p[2i + 1]) as floats.
 __device__ __forceinline__ void widen_i8_32(const uint4 (&u)[2], uint64_t (&P)[kPairs]) {
 #pragma unroll
@@ -159,20 +194,25 @@ __device__ __forceinline__ void widen_i8_32(const uint4 (&u)[2], uint64_t (&P)[k
 //   G == 64: bit 5 across lanes l and l ^ 1 (warp shuffle);
 //   G == 256: bits 5..7 after one exchange through shared memory: the 8 lanes
 //   of a group each write their 32 elements as 8 slots of 16 bytes and read
-//   slot t (elements 4t .. 4t + 3) of every lane of the group; slot m of lane
-//   s sits at 9 s + m (rows padded to 9 slots), so the 8 lanes of a
-//   quarter-warp (one group) hit 8 distinct bank quads on both sides, and every
-//   address is a per-lane base plus a constant.  Afterwards lane t holds in
-//   P[2 s + q] the elements (32 s + 4t + 2q, 32 s + 4t + 2q + 1), s = 0..7.
-constexpr int kXchGroupBytes = 8 * 9 * 16;
+//   slot t (elements 4t .. 4t + 3) of every lane of the group.  Slot m of
+//   lane s sits at 9 s + m (rows padded to 9 slots) and the groups are 1160
+//   bytes apart (8 more than their 72 slots), so the 64-bit halves that each
+//   access moves (a pair register, never a packed quad) hit 16 distinct bank
+//   pairs in every 16-lane phase, on both sides; every address is a per-lane
+//   base plus a constant.  Afterwards lane t holds in P[2 s + q] the elements
+//   (32 s + 4t + 2q, 32 s + 4t + 2q + 1), s = 0..7.
+constexpr int kXchGroupBytes = 8 * 9 * 16 + 8;
 constexpr int kXchBytesPerWarp = 4 * kXchGroupBytes;  // 4 groups
 
-template <int G>
+// kStage0 = false: bit 0 was already applied (widen_stage0_32).
+template <int G, bool kStage0 = true>
 __device__ __forceinline__ void fwht32(uint64_t (&P)[kPairs], uint32_t xch, uint32_t lane) {
+  if constexpr (kStage0) {
 #pragma unroll
-  for (int i = 0; i < kPairs; ++i) {  // bit 0
-    const float a = plo(P[i]), b = phi(P[i]);
-    P[i] = pk(a + b, a - b);
+    for (int i = 0; i < kPairs; ++i) {  // bit 0
+      const float a = plo(P[i]), b = phi(P[i]);
+      P[i] = pk(a + b, a - b);
+    }
   }
   constexpr int kTop = (G < kVec ? G : kVec) / 2;  // pair-index stages (bits 1..)
 #pragma unroll
@@ -201,10 +241,16 @@ __device__ __forceinline__ void fwht32(uint64_t (&P)[kPairs], uint32_t xch, uint
     const uint32_t g = xch + (lane >> 3) * kXchGroupBytes;
     const uint32_t wbase = g + 144 * t, rbase = g + 16 * t;
 #pragma unroll
-    for (int m = 0; m < 8; ++m) sts128(wbase + 16 * m, P[2 * m], P[2 * m + 1]);
+    for (int m = 0; m < 8; ++m) {
+      sts64(wbase + 16 * m, P[2 * m]);
+      sts64(wbase + 16 * m + 8, P[2 * m + 1]);
+    }
     __syncwarp();
 #pragma unroll
-    for (int s = 0; s < 8; ++s) lds128(rbase + 144 * s, P[2 * s], P[2 * s + 1]);
+    for (int s = 0; s < 8; ++s) {
+      P[2 * s] = lds64(rbase + 144 * s);
+      P[2 * s + 1] = lds64(rbase + 144 * s + 8);
+    }
     __syncwarp();
 #pragma unroll
     for (int h = 1; h < 8; h <<= 1) {  // bits 5..7: across source lanes
@@ -484,11 +530,11 @@ __global__ void __launch_bounds__(kMaxThreads, kMinBlocks) rotate_quant_act_hada
     __syncwarp();  // the lanes' copies landed: every lane's units are visible
     unstage_chunk<4>(rd_src, u);
     uint64_t P[kPairs];
-    widen16_32<kF16>(u, P);
+    widen_stage0_32<kF16>(u, P);
     __syncwarp();  // every lane has read its units before the slot is refilled
     src += src_step;
     stage_copies<4>(cp_dst, src, row + row_step < M ? lim : 0);
-    fwht32<G>(P, xch, lane);
+    fwht32<G, false>(P, xch, lane);
     float amax = warp_max(ok ? absmax32(P) : 0.f);
     if (team_warps > 1) {
       float* rb_red = red[it & 1];
