@@ -19,7 +19,7 @@ Entry points (same names as the C ABI, without the `convrot_` prefix; the
     linear_dequant(x, Wq, s_w, rot, bias)    -> y (the default path: decode, then dense_linear)
     linear_checked(x, Wq, s_w, rot, bias)    -> (y, path) (int8 compute, first call checked)
     check_state(device), check_reset(), check_set_min_cosine(t), check_min_cosine()
-    workspace_bytes(M, N, K), check_status(), selftest_wait_timeout(ms), measure_int8_mma_rate()
+    workspace_bytes(M, N, K), check_status(), selftest_wait_timeout(ms)
     ConvRotLinear(W, R, bias, mode)           the layer: forward, decode_weight
 """
 
@@ -39,7 +39,6 @@ __all__ = [
     "device_supported", "library_path", "ConvRotLinear", "linear_int8_noalloc",
     "noalloc_scratch_bytes", "selftest_wait_timeout", "dense_linear", "linear_dequant",
     "linear_checked", "check_state", "check_reset", "check_set_min_cosine", "check_min_cosine",
-    "measure_int8_mma_rate",
 ]
 
 OK, INVALID_ARG, UNSUPPORTED, CUDA, WORKSPACE, TIMEOUT, ALIGNMENT = range(7)
@@ -95,7 +94,6 @@ def _load() -> ctypes.CDLL:
         "convrot_check_reset": ([], None),
         "convrot_check_set_min_cosine": ([ctypes.c_double], i32),
         "convrot_check_min_cosine": ([], ctypes.c_double),
-        "convrot_measure_int8_mma_rate": ([i32, ctypes.POINTER(ctypes.c_double), vp], i32),
     }
     for f in ("", "_f16"):
         sigs["convrot_dense_linear" + f] = ([vp, i64, i64, i64, vp, vp, vp, vp], i32)
@@ -496,15 +494,6 @@ def check_set_min_cosine(threshold: float) -> None:
 
 def check_min_cosine() -> float:
     return float(_lib.convrot_check_min_cosine())
-
-
-def measure_int8_mma_rate(iters: int = 32768) -> float:
-    """Measured int8 tensor-core rate of the current device in TOP/s: every SM
-    issues back-to-back tcgen05.mma.kind::i8 on pseudo-random operands held in
-    shared memory (a burst of about 10 ms at the default `iters`)."""
-    tops = ctypes.c_double(0.0)
-    _check(_lib.convrot_measure_int8_mma_rate(int(iters), ctypes.byref(tops), _stream()))
-    return float(tops.value)
 
 
 def noalloc_scratch_bytes() -> int:

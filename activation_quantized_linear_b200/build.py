@@ -1,4 +1,5 @@
-"""Build libconvrot.so in place with nvcc for sm_100a.
+"""Build libconvrot.so (the layer) and libconvrot_bench.so (the benchmark's
+int8 tensor-core rate probe) in place with nvcc for sm_100a.
 
 Usage: python activation_quantized_linear_b200/build.py [--verbose] [--ptxas-info]
 (run as a script: importing the package loads the library it builds)
@@ -22,6 +23,8 @@ CSRC = os.path.join(PKG_DIR, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB_NAME = "libconvrot.so"
 LIB_PATH = os.path.join(PKG_DIR, LIB_NAME)
+BENCH_SRC = os.path.join(CSRC, "bench")
+BENCH_LIB_PATH = os.path.join(PKG_DIR, "libconvrot_bench.so")
 
 ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
@@ -37,24 +40,27 @@ def sources() -> list[str]:
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
 
 
+def bench_sources() -> list[str]:
+    return sorted(glob.glob(os.path.join(BENCH_SRC, "*.cu")))
+
+
 def needs_rebuild() -> bool:
-    if not os.path.exists(LIB_PATH):
+    if not os.path.exists(LIB_PATH) or not os.path.exists(BENCH_LIB_PATH):
         return True
-    t = os.path.getmtime(LIB_PATH)
-    deps = sources() + glob.glob(os.path.join(CSRC, "*.h")) + glob.glob(os.path.join(CSRC, "*.cuh"))
-    deps += glob.glob(os.path.join(INCLUDE, "*.h")) + [os.path.abspath(__file__)]
+    t = min(os.path.getmtime(LIB_PATH), os.path.getmtime(BENCH_LIB_PATH))
+    deps = sources() + bench_sources() + glob.glob(os.path.join(CSRC, "*.h"))
+    deps += glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(INCLUDE, "*.h"))
+    deps += [os.path.abspath(__file__)]
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) -> str:
-    if not force and not ptxas_info and not needs_rebuild():
-        return LIB_PATH
-    tmp = LIB_PATH + ".tmp"
+def _nvcc(srcs: list[str], out: str, verbose: bool, ptxas_info: bool) -> None:
+    tmp = out + ".tmp"
     cmd = [
         nvcc_path(), *ARCH_FLAGS, "-lineinfo", "-O3", "-std=c++17",
         "-Xcompiler", "-fPIC,-O3", "-shared", "-cudart", "static",
         "-I", INCLUDE, "-I", CSRC,
-        *sources(), "-o", tmp,
+        *srcs, "-o", tmp,
     ]
     if ptxas_info:
         cmd.insert(1, "-Xptxas=-v")
@@ -65,7 +71,14 @@ def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) 
         raise RuntimeError(f"nvcc failed ({res.returncode}):\n{res.stdout}\n{res.stderr}")
     if verbose or ptxas_info:
         sys.stdout.write(res.stdout + res.stderr)
-    os.replace(tmp, LIB_PATH)
+    os.replace(tmp, out)
+
+
+def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) -> str:
+    if not force and not ptxas_info and not needs_rebuild():
+        return LIB_PATH
+    _nvcc(sources(), LIB_PATH, verbose, ptxas_info)
+    _nvcc(bench_sources(), BENCH_LIB_PATH, verbose, ptxas_info)
     return LIB_PATH
 
 

@@ -3,6 +3,17 @@
 // measure on an RTX 4090; the denominator itself is the measured bf16 GEMM
 // rate times the nominal int8 : bf16 ratio of 2).
 //
+// Measurement tooling, not part of the layer: this file builds into its own
+// library (libconvrot_bench.so) that only the benchmark and its tests load;
+// the layer's library (libconvrot.so, include/convrot.h) does not export it.
+//
+// C entry point (plain int status, the convrot_status numbering):
+//   int convrot_bench_int8_mma_rate(int iters, double* tops, void* stream);
+//   iters in [1, 200000] (32768 runs for about 10 ms), else 1 (invalid
+//   argument, before any launch); 3 on a CUDA error; 5 if the kernel's
+//   bounded wait ran out; 0 with `tops` (a HOST pointer) set.  Synchronizes
+//   `stream` (a cudaStream_t, NULL for the legacy default stream).
+//
 // One CTA per SM issues back-to-back tcgen05.mma.kind::i8 instructions
 // (M = 128, N = 256, K = 32; the single-CTA form of the GEMM's instruction)
 // on operands that stay in shared memory, accumulating into one 256-column
@@ -12,11 +23,12 @@
 
 #include <cstdint>
 
-#include "internal.h"
 #include "sm100_ptx.cuh"
 
 namespace convrot {
 namespace {
+
+__device__ unsigned int g_probe_status;  // bit 0: the bounded wait ran out
 
 constexpr int kPeakThreads = 64;
 constexpr int kARows = 128, kBRows = 256, kRowBytes = 128;
@@ -81,16 +93,19 @@ __global__ void __launch_bounds__(kPeakThreads, 1)
   if (warp == 0) ptx::tmem_dealloc(tmem, kPeakTmemCols);
 }
 
-}  // namespace
-
-cudaError_t measure_int8_mma_rate(int iters, double* tops, cudaStream_t stream) {
+cudaError_t measure(int iters, double* tops, cudaStream_t stream) {
   unsigned int* status = nullptr;
-  cudaError_t e = status_word(&status);
+  cudaError_t e = cudaGetSymbolAddress(reinterpret_cast<void**>(&status), g_probe_status);
+  if (e != cudaSuccess) return e;
+  e = cudaMemsetAsync(status, 0, sizeof(unsigned int), stream);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(int8_mma_issue_loop, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(kPeakSmem));
   if (e != cudaSuccess) return e;
-  const int sms = sm_count();
+  int dev = 0, sms = 0;
+  e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
   cudaEvent_t e0, e1;
   e = cudaEventCreate(&e0);
   if (e != cudaSuccess) return e;
@@ -116,4 +131,14 @@ cudaError_t measure_int8_mma_rate(int iters, double* tops, cudaStream_t stream) 
   return cudaSuccess;
 }
 
+}  // namespace
 }  // namespace convrot
+
+extern "C" int convrot_bench_int8_mma_rate(int iters, double* tops, void* stream) {
+  if (tops == nullptr || iters < 1 || iters > 200000) return 1;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (convrot::measure(iters, tops, st) != cudaSuccess) return 3;
+  unsigned int status = 0;
+  if (cudaMemcpyFromSymbol(&status, convrot::g_probe_status, sizeof(status)) != cudaSuccess) return 3;
+  return (status & 1u) ? 5 : 0;
+}

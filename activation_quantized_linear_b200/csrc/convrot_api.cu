@@ -569,19 +569,6 @@ convrot_status convrot_selftest_wait_timeout(int limit_ms, convrot_stream_t stre
                   "selftest_wait_timeout launch");
 }
 
-convrot_status convrot_measure_int8_mma_rate(int iters, double* tops, convrot_stream_t stream) {
-  if (tops == nullptr) return fail(CONVROT_ERR_INVALID_ARG, "tops is NULL");
-  if (iters < 1 || iters > 200000) {
-    return fail(CONVROT_ERR_INVALID_ARG, "iters=%d must be in [1, 200000]", iters);
-  }
-  int dev = -1;
-  convrot_status s = current_device(&dev);
-  if (s != CONVROT_OK) return s;
-  cudaError_t e = convrot::measure_int8_mma_rate(iters, tops, as_stream(stream));
-  if (e != cudaSuccess) return cuda_fail(e, "measure_int8_mma_rate");
-  return convrot_check_status(stream);
-}
-
 convrot_status convrot_check_status(convrot_stream_t stream) {
   unsigned int st = 0;
   cudaError_t e = convrot::read_and_clear_status(&st, as_stream(stream));

@@ -72,11 +72,6 @@ cudaError_t launch_gemm16(const GemmArgs& a, cudaStream_t stream);
 // after `limit_ns` and records a timeout in the status word.
 cudaError_t launch_bounded_wait_selftest(uint64_t limit_ns, cudaStream_t stream);
 
-// Times one launch of the int8 MMA issue loop (every SM issues `iters` x 4
-// tcgen05.mma.kind::i8 of 128 x 256 x 32) and returns the rate in TOP/s.
-// Synchronizes `stream`.
-cudaError_t measure_int8_mma_rate(int iters, double* tops, cudaStream_t stream);
-
 // Reads and clears the current device's kernel status word (0 = fine).
 cudaError_t read_and_clear_status(unsigned int* status, cudaStream_t stream);
 

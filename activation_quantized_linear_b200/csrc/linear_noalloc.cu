@@ -12,10 +12,14 @@
 // static device memory instead, so the caller passes only inputs and outputs.
 //
 // The array lives in every GPU that loads the library, until the process
-// exits.  All calls share it and it keeps the previous call's contents; the
-// kernels overwrite every byte they read, so nothing needs clearing between
-// calls, but two calls that run at the same time on the GPU (different streams
-// or threads) race on it and must be serialized by the caller.
+// exits.  A batch whose codes do not fit it runs in row slices, as
+// convrot_linear_int8 does with a small workspace.  All calls share it and it
+// keeps the previous call's contents; the kernels overwrite every byte they
+// read, so nothing needs clearing between calls, but two calls that run at the
+// same time on the GPU (different streams or threads) race on it and must be
+// serialized by the caller.  Its device address is looked up once per device
+// and kept: after cudaDeviceReset the entry point must not be called again in
+// that process (the old address would be stale).
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -29,7 +33,8 @@ namespace {
 
 constexpr size_t kNoAllocScratchBytes = CONVROT_NOALLOC_SCRATCH_BYTES;
 
-// The scratch: int8 codes [M, K] at offset 0, per-token scales [M] after them.
+// The scratch: int8 codes [rows, K] at offset 0, per-token scales [rows] after
+// them (256-byte aligned), rows = as many tokens as fit.
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
 
 size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
@@ -68,13 +73,13 @@ extern "C" convrot_status convrot_linear_int8_noalloc(const convrot_bf16* x, int
     // M == 0 is a no-op; negative or empty sizes get the regular argument error.
     return convrot_linear_int8(x, M, K, N, R, Wq, s_w, s_w_len, bias, y, nullptr, 0, stream);
   }
-  const size_t need = round256(static_cast<size_t>(M) * static_cast<size_t>(K)) +
-                      round256(sizeof(float) * static_cast<size_t>(M));
+  // one token's codes and scale must fit; more tokens run in row slices
+  const size_t need = round256(static_cast<size_t>(K)) + round256(sizeof(float));
   if (need > kNoAllocScratchBytes) {
     return convrot::set_last_error(
         CONVROT_ERR_UNSUPPORTED,
-        "linear_int8_noalloc: M*K + 4*M (each rounded up to 256 B) = %zu bytes exceeds the "
-        "static scratch of %zu bytes; call convrot_linear_int8 with a workspace instead",
+        "linear_int8_noalloc: one token's codes and scale (%zu bytes) exceed the static "
+        "scratch of %zu bytes; call convrot_linear_int8 with a workspace instead",
         need, kNoAllocScratchBytes);
   }
   void* scratch = nullptr;

@@ -572,7 +572,7 @@ __host__ __device__ constexpr int flat_aux_bytes() {
 // kF16: the 16-bit float format of W (absmax / quant) or of W_hat (decode).
 template <int G, int MODE, bool PER_ROW_SCALE, bool kF16>
 __global__ void __launch_bounds__(256, MODE == kFlatDequant ? 3 : 4) hadamard_flat(const void* __restrict__ in, int64_t nchunks,
-                                                     int64_t chunks_per_row,
+                                                     uint64_t row_mul, int row_shift,
                                                      const float* __restrict__ scale,
                                                      void* __restrict__ out,
                                                      unsigned int* __restrict__ absmax_bits) {
@@ -642,7 +642,9 @@ __global__ void __launch_bounds__(256, MODE == kFlatDequant ? 3 : 4) hadamard_fl
         }
       }
     } else {
-      const float sw = PER_ROW_SCALE ? scale[(ok ? c : 0) / chunks_per_row] : scale[0];
+      // output row of chunk c: c / (K / 32) as a multiply and shift (row_reciprocal)
+      const float sw =
+          PER_ROW_SCALE ? scale[((ok ? static_cast<uint64_t>(c) : 0ull) * row_mul) >> row_shift] : scale[0];
       uint32_t w[kPairs];
       products16_32<kF16>(w, P, sw * norm);
       if constexpr (G == 256) {
@@ -887,6 +889,18 @@ cudaError_t rqa_hadamard(const uint16_t* x, int64_t M, int64_t K, int8_t* xq, fl
   return rqa_launch<G, 1024, 1, kF16>(x, M, k, team_warps, rows_per_cta, xq, s_tok, stream);
 }
 
+// Multiplier m and shift k with floor(c * m / 2^k) == c / d for every
+// 0 <= c < 2^31 (1 <= d < 2^31): k = 31 + ceil(log2 d), m = ceil(2^k / d).  With
+// e = m d - 2^k < d, c m / 2^k = c / d + c e / (d 2^k), and the second term is
+// below 2^31 / 2^k = 2^-ceil(log2 d) <= 1 / d, too small to carry c / d past
+// the next integer.
+void row_reciprocal(uint64_t d, uint64_t* m, int* k) {
+  int l = 0;
+  while ((1ull << l) < d) ++l;
+  *k = 31 + l;
+  *m = ((1ull << *k) + d - 1) / d;
+}
+
 template <int G, int MODE, bool PER_ROW, bool kF16>
 cudaError_t flat_launch(const void* in, int64_t nchunks, int64_t chunks_per_row,
                         const float* scale, void* out, unsigned int* absmax_bits,
@@ -904,8 +918,15 @@ cudaError_t flat_launch(const void* in, int64_t nchunks, int64_t chunks_per_row,
   int64_t grid = (nchunks + kThreadsFlat - 1) / kThreadsFlat;
   if (grid > cap) grid = cap;
   if (grid < 1) grid = 1;
+  uint64_t row_mul = 0;
+  int row_shift = 0;
+  if (PER_ROW) {
+    // the reciprocal is exact below 2^31 chunks (64 G weights: beyond any HBM)
+    if (nchunks >= (1ll << 31) || chunks_per_row < 1) return cudaErrorInvalidValue;
+    row_reciprocal(static_cast<uint64_t>(chunks_per_row), &row_mul, &row_shift);
+  }
   return launch_chained(hadamard_flat<G, MODE, PER_ROW, kF16>, grid, kThreadsFlat, smem, stream, in,
-                        nchunks, chunks_per_row, scale, out, absmax_bits);
+                        nchunks, row_mul, row_shift, scale, out, absmax_bits);
 }
 
 template <int G, typename TIn, int MODE, bool kF16>

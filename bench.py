@@ -421,7 +421,7 @@ def run_ours(args, lins):
     tops_frac = gemm_tops / int8_peak
     # the tensor cores' own int8 rate on this GPU (after the timed region):
     # context for the denominator, which stays the measured bf16 rate x 2
-    issue_tops = issue_loop_tops(cr)
+    issue_tops = issue_loop_tops()
     out = {
         "metric": "int8 ConvRot linear TOPS (rotate+quant+GEMM)",
         "value": value, "unit": "TOPS", "n_gpus": world, "steps": args.steps,
@@ -583,12 +583,41 @@ def run_sweep(args):
     return 0
 
 
-def issue_loop_tops(cr):
+class Int8RateProbe:
+    """The int8 tensor-core issue-rate probe: its own library
+    (libconvrot_bench.so, built beside the layer's), which the layer's
+    library does not export.  measure_int8_mma_rate(iters) -> TOP/s of one
+    launch in which every SM issues iters x 4 tcgen05.mma.kind::i8 of
+    128 x 256 x 32 on operands held in shared memory."""
+
+    def __init__(self):
+        import ctypes
+
+        from activation_quantized_linear_b200 import build
+        self._lib = ctypes.CDLL(build.BENCH_LIB_PATH)
+        f = self._lib.convrot_bench_int8_mma_rate
+        f.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_double), ctypes.c_void_p]
+        f.restype = ctypes.c_int
+        self._f = f
+
+    def measure_int8_mma_rate(self, iters: int = 32768) -> float:
+        import ctypes
+
+        import torch
+        tops = ctypes.c_double(0.0)
+        st = self._f(int(iters), ctypes.byref(tops), torch.cuda.current_stream().cuda_stream)
+        if st != 0:
+            raise RuntimeError(f"int8 issue-rate probe failed with status {st}")
+        return float(tops.value)
+
+
+def issue_loop_tops(probe=None):
     """The int8 tensor cores' measured burst rate (TOP/s), or None if the
     measurement fails: it is context for the roofline, never a reason to
     lose the bench line."""
     try:
-        return cr.measure_int8_mma_rate(32768)
+        probe = probe if probe is not None else Int8RateProbe()
+        return probe.measure_int8_mma_rate(32768)
     except Exception as exc:  # noqa: BLE001
         print(f"int8 issue-rate measurement failed: {exc}", file=sys.stderr)
         return None
@@ -659,7 +688,7 @@ def run_default_path(args):
                      "dense16_tflops": flops / t_dense / 1e9,
                      "dense16_frac_bf16_peak": flops / t_dense / 1e9 / bf16_tflops, **intmm})
         del Wq, W_hat, ws_i8, ws_dq, y
-    issue_tops = issue_loop_tops(cr)
+    issue_tops = issue_loop_tops()
     total_i8 = sum(r["int8_ms"] for r in rows)
     total_dq = sum(r["dequant_ms"] for r in rows)
     print(json.dumps({"compare": "int8_compute_vs_default_path", "workload": args.workload,

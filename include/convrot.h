@@ -26,9 +26,9 @@
  *     owns only the device copy of R inside a rotation handle.  No entry point
  *     allocates device memory, except convrot_rotation_create.
  *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL means the
- *     legacy default stream), except three that synchronize it and say so:
- *     convrot_check_status, the first call of a key in
- *     convrot_linear_checked, and convrot_measure_int8_mma_rate.  Argument errors return at once, before any
+ *     legacy default stream), except two that synchronize it and say so:
+ *     convrot_check_status and the first call of a key in
+ *     convrot_linear_checked.  Argument errors return at once, before any
  *     launch, and leave the outputs untouched.  A launch failure returns
  *     CONVROT_ERR_CUDA.  A wait inside a kernel that runs out of time (about a
  *     second) makes that kernel stop and record CONVROT_ERR_TIMEOUT in a device
@@ -181,10 +181,15 @@ convrot_status convrot_linear_int8(const convrot_bf16* x, int64_t M, int64_t K, 
  * codes and per-token scales in a static device array of
  * CONVROT_NOALLOC_SCRATCH_BYTES (32 MiB) that every GPU loading the library
  * holds until the process exits.  It allocates nothing itself.
- *   - Limit: round256(M*K) + round256(4*M) <= CONVROT_NOALLOC_SCRATCH_BYTES,
- *     else CONVROT_ERR_UNSUPPORTED with a message naming both sizes.
+ *   - Tokens whose codes and scales (round256(rows*K) + round256(4*rows)
+ *     bytes) do not fit the array at once run in row slices, one after the
+ *     other, with the same result.  Only a single token too large for it
+ *     (round256(K) + 256 > CONVROT_NOALLOC_SCRATCH_BYTES, beyond any K the
+ *     rotation accepts) is CONVROT_ERR_UNSUPPORTED.
  *   - The first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *     (cudaGetSymbolAddress) and keeps it; make that first call before any
+ *     stream capture, and do not call this entry point again after
+ *     cudaDeviceReset in the same process (the kept address would be stale).
  *   - All calls share the array: calls that overlap on the GPU (other streams,
  *     other host threads) race and must be serialized by the caller.  Each call
  *     overwrites all of the scratch it reads, so nothing is carried over.
@@ -341,19 +346,6 @@ convrot_status convrot_check_status(convrot_stream_t stream);
  * and the context stays usable.
  */
 convrot_status convrot_selftest_wait_timeout(int limit_ms, convrot_stream_t stream);
-
-/*
- * Measured int8 tensor-core rate of the current device, in TOP/s (no
- * counterpart on the pages: a cross-check for the int8 GEMM's roofline
- * denominator).  Every SM issues `iters` x 4 back-to-back
- * tcgen05.mma.kind::i8 of 128 x 256 x 32 on operands of pseudo-random bytes
- * held in shared memory, with nothing loaded or stored; one launch is timed
- * with CUDA events.
- * iters in [1, 200000] (32768 runs for about 10 ms), else
- * CONVROT_ERR_INVALID_ARG.  Synchronizes `stream`; `tops` is a HOST pointer.
- * Returns CONVROT_ERR_TIMEOUT if the kernel's bounded wait ran out.
- */
-convrot_status convrot_measure_int8_mma_rate(int iters, double* tops, convrot_stream_t stream);
 
 /* Message of the last failure on the calling thread ("" if none). */
 const char* convrot_last_error_string(void);

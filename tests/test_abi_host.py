@@ -146,9 +146,18 @@ def test_checked_rejects_before_device():
     assert cr.check_state(0) == (False, 0)
 
 
-def test_mma_rate_rejects_before_device():
+def test_bench_probe_is_its_own_library():
+    """The int8 issue-rate probe lives in libconvrot_bench.so, which the
+    benchmark loads; the layer's library does not export it.  Its argument
+    checks answer before any device work."""
+    raw = ctypes.CDLL(build.LIB_PATH)
+    assert not hasattr(raw, "convrot_measure_int8_mma_rate")
+    assert not hasattr(raw, "convrot_bench_int8_mma_rate")
+    probe = ctypes.CDLL(build.BENCH_LIB_PATH)
+    f = probe.convrot_bench_int8_mma_rate
+    f.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_double), ctypes.c_void_p]
+    f.restype = ctypes.c_int
     tops = ctypes.c_double(0.0)
-    f = lib.convrot_measure_int8_mma_rate
     assert f(0, ctypes.byref(tops), None) == cr.INVALID_ARG
     assert f(200001, ctypes.byref(tops), None) == cr.INVALID_ARG
     assert f(100, None, None) == cr.INVALID_ARG

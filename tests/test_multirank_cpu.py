@@ -86,5 +86,5 @@ def test_issue_loop_measurement_failure_keeps_the_bench_line():
             assert iters == 32768
             return 4321.0
 
-    assert bench.issue_loop_tops(Failing) is None
-    assert bench.issue_loop_tops(Working) == 4321.0
+    assert bench.issue_loop_tops(Failing()) is None
+    assert bench.issue_loop_tops(Working()) == 4321.0

@@ -71,18 +71,21 @@ def test_noalloc_matches_workspace_entry_point_two_calls():
     cr.check_status()
 
 
-def test_noalloc_rejects_problems_beyond_its_scratch():
+def test_noalloc_slices_batches_beyond_its_scratch():
+    """4608 tokens of K = 10240 need 47 MB of codes, more than the 32 MiB
+    array: the entry point runs them in row slices and still returns the
+    workspace entry point's output, bit for bit, on two calls in a row."""
     import activation_quantized_linear_b200 as cr
     torch.cuda.set_device(0)
     lib = cr._lib
-    rot = cr.Rotation(workloads.sylvester_rotation(256))
-    M, K, N = 4608, 10240, 64  # 47 MB of codes > 32 MiB
-    x = torch.zeros((M, K), dtype=torch.bfloat16, device="cuda")
-    Wq = torch.zeros((N, K), dtype=torch.int8, device="cuda")
-    s_w = torch.ones(1, device="cuda")
-    bias = torch.zeros(N, dtype=torch.bfloat16, device="cuda")
-    y = torch.zeros((M, N), dtype=torch.bfloat16, device="cuda")
-    st = _call_noalloc(lib, x, Wq, s_w, rot, bias, y)
-    assert st == cr.UNSUPPORTED
-    assert b"exceeds the static scratch" in lib.convrot_last_error_string()
-    assert not y.any()  # nothing was launched
+    lin = workloads.WORKLOADS["zimage_dit_block"][2]  # 4608 x 10240 -> 3840
+    assert lin.M * lin.K > lib.convrot_noalloc_scratch_bytes()
+    x, Wq, s_w, bias, rot = _layer(lin, 5)
+    y_ref = _call_with_workspace(cr, x, Wq, s_w, rot, bias)
+    for _ in range(2):
+        y = torch.full((x.shape[0], Wq.shape[0]), float("nan"), dtype=torch.bfloat16, device="cuda")
+        st = _call_noalloc(lib, x, Wq, s_w, rot, bias, y)
+        assert st == cr.OK, lib.convrot_last_error_string()
+        torch.cuda.synchronize()
+        assert torch.equal(y.view(torch.int16), y_ref.view(torch.int16))
+    cr.check_status()
