@@ -227,9 +227,27 @@ __device__ __forceinline__ void gemm_pair(const CUtensorMap& tmA, const CUtensor
   ptx::tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
   const int num_tiles = p.m_tiles * p.n_tiles;
-  // the set-up above overlaps the previous kernel of the stream; every global
-  // access below comes after it (the whole grid is resident, so the next
-  // kernel may be scheduled right away)
+  // The int8 weight (B) is never written by the kernel this one is chained
+  // to (nothing in this library writes int8 weights in a chained launch: the
+  // weight quantizer ends with a plain launch), so the producer issues the
+  // weight loads of its first stages before waiting on that kernel; they fill
+  // the ring while it drains.  The 16-bit GEMM's B is the decoded weight,
+  // which the decode right before it writes, so it waits first.
+  constexpr bool kEarlyB = kKind == kKindI8;
+  int early = 0;  // stages of the first tile whose B load is already issued
+  if (kEarlyB && threadIdx.x == 0 && unit < num_tiles) {
+    int mb, nb;
+    tile_coords(unit, p.m_tiles, p.n_tiles, p.group_m, mb, nb);
+    const int b_row = nb * BN + static_cast<int>(rank) * C::kBRows;
+    early = p.num_kb < C::kStages ? p.num_kb : C::kStages;
+    for (int kb = 0; kb < early; ++kb) {  // fresh ring: every stage is free
+      if (leader) ptx::mbar_arrive_expect_tx(&bars->full[kb], C::kTxBytes);
+      ptx::tma_load_2d_pair(sB + kb * C::kBStage, &tmB, &bars->full[kb], kb * KC::kStageK, b_row);
+    }
+  }
+  // the set-up above overlaps the previous kernel of the stream; every other
+  // global access below comes after it (the whole grid is resident, so the
+  // next kernel may be scheduled right away)
   ptx::grid_dependency_wait();
   ptx::grid_dependents_launch();
 
@@ -239,12 +257,25 @@ __device__ __forceinline__ void gemm_pair(const CUtensorMap& tmA, const CUtensor
     uint32_t phase = 0;
     int last_stage = -1;
     uint32_t last_phase = 0;
+    if (early > 0) {
+      // the first tile's early stages: their B is in flight, add A (always,
+      // so that every issued stage completes before the CTA can exit)
+      int mb, nb;
+      tile_coords(unit, p.m_tiles, p.n_tiles, p.group_m, mb, nb);
+      const int a_row = mb * C::kTileM + static_cast<int>(rank) * BM;
+      for (int kb = 0; kb < early; ++kb) {
+        ptx::tma_load_2d_pair(sA + kb * A_STAGE, &tmA, &bars->full[kb], kb * KC::kStageK, a_row);
+      }
+      last_stage = early - 1;
+      stage = early == C::kStages ? 0 : early;
+      phase = early == C::kStages ? 1u : 0u;
+    }
     for (int tile = unit; tile < num_tiles && !*abort_flag; tile += units) {
       int mb, nb;
       tile_coords(tile, p.m_tiles, p.n_tiles, p.group_m, mb, nb);
       const int a_row = mb * C::kTileM + static_cast<int>(rank) * BM;
       const int b_row = nb * BN + static_cast<int>(rank) * C::kBRows;
-      for (int kb = 0; kb < p.num_kb; ++kb) {
+      for (int kb = tile == unit ? early : 0; kb < p.num_kb; ++kb) {
         if (!wait_bounded(&bars->empty[stage], phase ^ 1u)) {
           record_timeout(abort_flag, p.status);
           break;

@@ -59,12 +59,18 @@ struct SkinnyCfg {
   // epilogue factors staged during the mainloop: s_tok of the NT tokens, s_w
   // and bias of the block's rows (f32)
   static constexpr int kEpiBytes = (NT + 2 * kRows) * 4;
-  // as many stages as fit (a CTA's whole K range in flight at once); the int32
-  // partial reuses the ring once the mainloop has drained it
-  static constexpr int kFit = (232448 - 1024 - 256 - kEpiBytes) / kStageBytes;
-  static constexpr int kStages = kFit > 12 ? 12 : kFit;
   static constexpr int kPartStride = NT + 4;  // int32 per partial row (padded: no bank conflicts)
   static constexpr int kPartBytes = kRows * kPartStride * 4;
+  // Two CTAs per SM when the ring that fits half of the SM's shared memory
+  // still holds the int32 partial and the peers' slices (NT <= 64): a CTA of
+  // the next launch then lands beside one of this launch, issues its weight
+  // loads while this one finishes, and a weight of more 128-row blocks than
+  // SMs runs in one wave.  Otherwise as many stages as fit one CTA per SM.
+  // The partial reuses the ring once the mainloop has drained it.
+  static constexpr int kHalfFit = (115712 - 1024 - 256 - kEpiBytes) / kStageBytes;
+  static constexpr int kFit = (232448 - 1024 - 256 - kEpiBytes) / kStageBytes;
+  static constexpr bool kTwoPerSm = 2 * kPartBytes <= kHalfFit * kStageBytes;
+  static constexpr int kStages = kTwoPerSm ? kHalfFit : (kFit > 12 ? 12 : kFit);
   // the partial and, after it, the slices the peers push (one per rank)
   static_assert(2 * kPartBytes <= kStages * kStageBytes, "partial and slices must fit in the ring");
   static constexpr size_t kSmem = 1024 + kStages * kStageBytes + 256 + kEpiBytes;
@@ -83,7 +89,7 @@ struct SkinnyBars {
 };
 
 template <int NT>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, SkinnyCfg<NT>::kTwoPerSm ? 2 : 1)
     int8_gemm_skinny(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                      const SkinnyParams p) {
   using C = SkinnyCfg<NT>;
@@ -131,16 +137,31 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
-  // the set-up above overlaps the previous kernel of the stream; every global
-  // access below comes after it
+  // The int8 weight is never written by the kernel this one is chained to
+  // (the library's weight quantizer ends with a plain launch), so the
+  // producer issues the weight loads of its first stages before waiting on
+  // that kernel: they stream while it drains.  The tokens' codes come after.
+  const int early = kb1 - kb0 < kStages ? (kb1 > kb0 ? kb1 - kb0 : 0) : kStages;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < early; ++i) {  // fresh ring: every stage is free
+      ptx::mbar_arrive_expect_tx(&bars->full[i], C::kStageBytes);
+      ptx::tma_load_2d(sA + i * C::kAStage, &tmW, &bars->full[i], (kb0 + i) * kBK, block * kRows);
+    }
+  }
+  // the set-up above overlaps the previous kernel of the stream; every other
+  // global access below comes after it
   ptx::grid_dependency_wait();
   ptx::grid_dependents_launch();
 
   if (threadIdx.x == 0) {
     // ------------------------------------------------------------ producer
-    int stage = 0;
-    uint32_t phase = 0;
-    for (int kb = kb0; kb < kb1; ++kb) {
+    // the early stages' codes first (always, so every issued stage completes)
+    for (int i = 0; i < early; ++i) {
+      ptx::tma_load_2d(sB + i * C::kBStage, &tmX, &bars->full[i], (kb0 + i) * kBK, 0);
+    }
+    int stage = early == kStages ? 0 : early;
+    uint32_t phase = early == kStages ? 1u : 0u;
+    for (int kb = kb0 + early; kb < kb1; ++kb) {
       if (!ptx::mbar_wait(&bars->empty[stage], phase ^ 1u, ptx::globaltimer_ns() + kWaitNs)) {
         atomicOr(p.status, 1u);
         *abort_flag = 1;
@@ -210,7 +231,43 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::tc_fence_after();
     const uint32_t t_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     int32_t* dst = part + row * C::kPartStride;
-    if (kb1 <= kb0 || !ready || *abort_flag) {
+    if (p.splits == 1) {
+      // one CTA holds the whole K: each thread drains its weight row n from
+      // TMEM straight to y[:, n] (a warp's 32 rows are 32 consecutive outputs
+      // of a token); the factors staged above are read after the four
+      // epilogue warps' barrier, which every one of them reaches.  After a
+      // timeout nothing is stored (the status word reports it).
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      const bool drain = ready && !__any_sync(0xffffffffu, *abort_flag != 0);
+      const int64_t n = static_cast<int64_t>(block) * kRows + row;
+      const float sw = p.out_s32 ? 0.f : ep_sw[row];
+      const float bn = p.out_s32 ? 0.f : ep_bias[row];
+#pragma unroll 1
+      for (int c0 = 0; drain && c0 < NT; c0 += 16) {
+        uint32_t r[16];
+        ptx::tmem_ld_32x32b_x16(t_base + c0, r);
+        ptx::tmem_ld_wait();
+        if (n >= p.N) continue;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const int64_t m = c0 + j;
+          if (m >= p.M) break;
+          if (p.out_s32) {
+            static_cast<int32_t*>(p.out)[m * p.N + n] = static_cast<int32_t>(r[j]);
+          } else {
+            const float y = fmaf(__int2float_rn(static_cast<int32_t>(r[j])), ep_tok[m] * sw, bn);
+            uint16_t bits;
+            if (p.out_f16) {
+              bits = __half_as_ushort(__float2half_rn(y));
+            } else {
+              const __nv_bfloat16 h = __float2bfloat16_rn(y);
+              bits = *reinterpret_cast<const uint16_t*>(&h);
+            }
+            static_cast<uint16_t*>(p.out)[m * p.N + n] = bits;
+          }
+        }
+      }
+    } else if (kb1 <= kb0 || !ready || *abort_flag) {
       if (!ready && lane == 0) atomicOr(p.status, 1u);
 #pragma unroll
       for (int c = 0; c < NT; c += 4) *reinterpret_cast<int4*>(dst + c) = make_int4(0, 0, 0, 0);
@@ -264,7 +321,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // copy out of this CTA has too, and its shared memory may be released
   __syncwarp();
   ptx::cluster_arrive();
-  {
+  if (p.splits > 1) {
     // (row, 4 tokens) items; consecutive threads take consecutive weight rows
     const int items = rows * (NT / 4);
     for (int it = threadIdx.x; it < items; it += kThreads) {
@@ -331,7 +388,7 @@ cudaError_t launch_nt(const GemmArgs& a, SkinnyParams p, cudaStream_t stream) {
                                        static_cast<int>(C::kSmem));
   if (e != cudaSuccess) return e;
   const int blocks = static_cast<int>((a.N + kRows - 1) / kRows);
-  int splits = sm_count() / blocks;  // one wave of CTAs
+  int splits = sm_count() / blocks;  // one CTA per SM, one wave
   splits = splits < 1 ? 1 : (splits > 8 ? 8 : splits);
   if (splits > p.num_kb) splits = p.num_kb;
   while (kRows % splits) --splits;  // each rank finishes an equal share of the 128 rows
