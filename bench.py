@@ -42,8 +42,15 @@ INT8_PER_BF16 = 2.0  # nominal dense int8 : bf16 tensor throughput (4.5 : 2.25 P
 # DRAM bytes per launch from ncu (dram__bytes_read.sum + dram__bytes_write.sum),
 # averaged over the GEMM launches of one step of a workload, valid only for the
 # kernel source they were taken on (first 16 hex digits of its sha256).
-NCU_TRAFFIC = {("int8_gemm_tcgen05", "zimage_dit_block"): (120.24e6 + 102.27e6 + 151.76e6) / 3}
-NCU_TRAFFIC_SOURCE_SHA = {("int8_gemm_tcgen05", "zimage_dit_block"): "401d1e52793f0ba8"}
+NCU_TRAFFIC = {
+    ("int8_gemm_tcgen05", "zimage_dit_block"): (120.24e6 + 102.27e6 + 151.76e6) / 3,
+    ("int8_gemm_tcgen05", "wan22_a14b_video_dit"):
+        ((166.00e6 + 210.10e6) + (156.76e6 + 187.52e6) + (557.14e6 + 70.09e6)) / 3,
+}
+NCU_TRAFFIC_SOURCE_SHA = {
+    ("int8_gemm_tcgen05", "zimage_dit_block"): "401d1e52793f0ba8",
+    ("int8_gemm_tcgen05", "wan22_a14b_video_dit"): "4f103f468a403a96",
+}
 
 
 def source_sha(rel: str) -> str:
@@ -520,19 +527,23 @@ def run_sweep(args):
     # few tokens, launched back to back as in a model (chained launches), each
     # launch on its own weight copy so that the weights (8 x 16.8 MB) stream
     # from HBM, not L2
+    # K = N = 4096 and the few-token forms of the workloads' wide and deep
+    # linears (FLUX.1 fused in-projection, Z-Image QKV and FFN down)
     chained = []
     rot = cr.Rotation(workloads.sylvester_rotation(256))
-    Ws = [torch.randint(-127, 128, (4096, 4096), dtype=torch.int8, device="cuda") for _ in range(8)]
     sw1 = torch.tensor([1e-3], device="cuda")
-    for Mc in (1, 16, 64, 128):
-        xq = torch.randint(-127, 128, (Mc, 4096), dtype=torch.int8, device="cuda")
-        st = torch.rand(Mc, device="cuda") * 1e-3
-        y = torch.empty((Mc, 4096), dtype=torch.bfloat16, device="cuda")
-        t = timed(lambda: [cr.int8_gemm(xq, st, W, sw1, None, out=y) for W in Ws], args.steps) / len(Ws)
-        wbytes = Mc * 4096 + 4096 * 4096 + 2 * Mc * 4096
-        chained.append({"M": Mc, "gemm_ms": t, "gemm_GBps": wbytes / t / 1e6,
-                        "gemm_frac_hbm": wbytes / t / 1e6 / hbm_gbs})
-    del Ws
+    for Kc, Nc, copies in ((4096, 4096, 8), (3072, 21504, 3), (3840, 11520, 4), (10240, 3840, 4)):
+        Ws = [torch.randint(-127, 128, (Nc, Kc), dtype=torch.int8, device="cuda") for _ in range(copies)]
+        for Mc in (1, 16, 64, 128):
+            xq = torch.randint(-127, 128, (Mc, Kc), dtype=torch.int8, device="cuda")
+            st = torch.rand(Mc, device="cuda") * 1e-3
+            y = torch.empty((Mc, Nc), dtype=torch.bfloat16, device="cuda")
+            t = timed(lambda: [cr.int8_gemm(xq, st, W, sw1, None, out=y) for W in Ws],
+                      args.steps) / len(Ws)
+            wbytes = Mc * Kc + Nc * Kc + 2 * Mc * Nc
+            chained.append({"K": Kc, "N": Nc, "M": Mc, "gemm_ms": t, "gemm_GBps": wbytes / t / 1e6,
+                            "gemm_frac_hbm": wbytes / t / 1e6 / hbm_gbs})
+        del Ws
     # per-output-channel weight scales and fp16 activations/outputs, G = 256:
     # the GEMM at M = 8192 and the [12288, 3072] decode
     var = []
