@@ -41,12 +41,12 @@ __all__ = [
     "linear_checked", "check_state", "check_reset", "check_set_min_cosine", "check_min_cosine",
 ]
 
-OK, INVALID_ARG, UNSUPPORTED, CUDA, WORKSPACE, TIMEOUT, ALIGNMENT = range(7)
+OK, INVALID_ARG, UNSUPPORTED, CUDA, WORKSPACE, TIMEOUT, ALIGNMENT, BOUNDS = range(8)
 OP_LINEAR_INT8, OP_LINEAR_INT8_SLICED, OP_LINEAR_DEQUANT, OP_LINEAR_CHECKED = 1, 2, 3, 4
 PATH_INT8, PATH_DEQUANT = 1, 2
 CHECK_ROWS = 256
 STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "CUDA", 4: "WORKSPACE",
-                5: "TIMEOUT", 6: "ALIGNMENT"}
+                5: "TIMEOUT", 6: "ALIGNMENT", 7: "BOUNDS"}
 
 
 class ConvRotError(RuntimeError):
@@ -59,8 +59,9 @@ def library_path() -> str:
     return _build.LIB_PATH
 
 
-def _load() -> ctypes.CDLL:
-    path = _build.LIB_PATH
+def load_library(path: str) -> ctypes.CDLL:
+    """libconvrot.so, or a library built from the same sources (the debug
+    library, build.DEBUG_LIB_PATH), with the C signatures of include/convrot.h."""
     if not os.path.exists(path):
         raise ImportError(
             f"{path} is missing: build it with `python activation_quantized_linear_b200/build.py`"
@@ -108,7 +109,7 @@ def _load() -> ctypes.CDLL:
     return lib
 
 
-_lib = _load()
+_lib = load_library(_build.LIB_PATH)
 
 
 def _check(status: int) -> None:

@@ -1,5 +1,7 @@
-"""Build libconvrot.so (the layer) and libconvrot_bench.so (the benchmark's
-int8 tensor-core rate probe) in place with nvcc for sm_100a.
+"""Build, in place with nvcc for sm_100a: libconvrot.so (the layer),
+libconvrot_debug.so (the same sources with CONVROT_DEBUG=1: device-side
+bounds checks and the tests' fault injection, include/convrot_debug.h) and
+libconvrot_bench.so (the benchmark's int8 tensor-core rate probe).
 
 Usage: python activation_quantized_linear_b200/build.py [--verbose] [--ptxas-info]
 (run as a script: importing the package loads the library it builds)
@@ -25,6 +27,7 @@ LIB_NAME = "libconvrot.so"
 LIB_PATH = os.path.join(PKG_DIR, LIB_NAME)
 BENCH_SRC = os.path.join(CSRC, "bench")
 BENCH_LIB_PATH = os.path.join(PKG_DIR, "libconvrot_bench.so")
+DEBUG_LIB_PATH = os.path.join(PKG_DIR, "libconvrot_debug.so")
 
 ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
@@ -45,21 +48,22 @@ def bench_sources() -> list[str]:
 
 
 def needs_rebuild() -> bool:
-    if not os.path.exists(LIB_PATH) or not os.path.exists(BENCH_LIB_PATH):
+    libs = (LIB_PATH, BENCH_LIB_PATH, DEBUG_LIB_PATH)
+    if not all(os.path.exists(p) for p in libs):
         return True
-    t = min(os.path.getmtime(LIB_PATH), os.path.getmtime(BENCH_LIB_PATH))
+    t = min(os.path.getmtime(p) for p in libs)
     deps = sources() + bench_sources() + glob.glob(os.path.join(CSRC, "*.h"))
     deps += glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(INCLUDE, "*.h"))
     deps += [os.path.abspath(__file__)]
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def _nvcc(srcs: list[str], out: str, verbose: bool, ptxas_info: bool) -> None:
+def _nvcc(srcs: list[str], out: str, verbose: bool, ptxas_info: bool, defines=()) -> None:
     tmp = out + ".tmp"
     cmd = [
         nvcc_path(), *ARCH_FLAGS, "-lineinfo", "-O3", "-std=c++17",
         "-Xcompiler", "-fPIC,-O3", "-shared", "-cudart", "static",
-        "-I", INCLUDE, "-I", CSRC,
+        "-I", INCLUDE, "-I", CSRC, *defines,
         *srcs, "-o", tmp,
     ]
     if ptxas_info:
@@ -78,6 +82,7 @@ def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) 
     if not force and not ptxas_info and not needs_rebuild():
         return LIB_PATH
     _nvcc(sources(), LIB_PATH, verbose, ptxas_info)
+    _nvcc(sources(), DEBUG_LIB_PATH, verbose, ptxas_info, defines=("-DCONVROT_DEBUG=1",))
     _nvcc(bench_sources(), BENCH_LIB_PATH, verbose, ptxas_info)
     return LIB_PATH
 

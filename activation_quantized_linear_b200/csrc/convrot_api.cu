@@ -12,6 +12,7 @@
 #include <vector>
 
 #include "convrot.h"
+#include "convrot_debug.h"
 #include "internal.h"
 
 namespace {
@@ -573,8 +574,24 @@ convrot_status convrot_check_status(convrot_stream_t stream) {
   unsigned int st = 0;
   cudaError_t e = convrot::read_and_clear_status(&st, as_stream(stream));
   if (e != cudaSuccess) return cuda_fail(e, "convrot_check_status");
-  if (st & 1u) return fail(CONVROT_ERR_TIMEOUT, "a kernel gave up a bounded wait (timeout)");
+  if (st & convrot::kStatusTimeout) {
+    return fail(CONVROT_ERR_TIMEOUT, "a kernel gave up a bounded wait (timeout)");
+  }
+  if (st & convrot::kStatusBounds) {
+    return fail(CONVROT_ERR_BOUNDS, "a kernel caught an out-of-range index and skipped it (debug build)");
+  }
   return CONVROT_OK;
 }
+
+#if CONVROT_DEBUG
+convrot_status convrot_debug_set_fault(int fault) {
+  if (fault != CONVROT_FAULT_NONE && fault != CONVROT_FAULT_SKIP_STAGE &&
+      fault != CONVROT_FAULT_SHORT_ROWS) {
+    return fail(CONVROT_ERR_INVALID_ARG, "unknown fault %d", fault);
+  }
+  convrot::set_debug_fault(fault);
+  return CONVROT_OK;
+}
+#endif
 
 }  // extern "C"

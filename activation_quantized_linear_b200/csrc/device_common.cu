@@ -3,6 +3,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstring>
 #include <mutex>
 #include <vector>
@@ -52,6 +53,13 @@ bool encode_tma_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+
+namespace {
+std::atomic<int> g_debug_fault{0};  // only the debug library's test hook sets it
+}  // namespace
+
+int debug_fault() { return CONVROT_DEBUG ? g_debug_fault.load() : 0; }
+void set_debug_fault(int code) { g_debug_fault.store(code); }
 
 int sm_count() {
   static std::mutex mu;

@@ -90,7 +90,8 @@ struct Params {
   int per_channel_scale;
   int out_s32;
   int out_f16;           // y and bias fp16 (else bf16)
-  unsigned int* status;  // device status word (bit 0: a wait ran out)
+  unsigned int* status;  // device status word (bit 0: a wait ran out; bit 1: debug bounds)
+  int fault;             // debug build: injected fault (kFaultSkipStage, kFaultShortRows)
 };
 
 template <int STAGES>
@@ -234,6 +235,10 @@ __device__ __forceinline__ void gemm_pair(const CUtensorMap& tmA, const CUtensor
   // the ring while it drains.  The 16-bit GEMM's B is the decoded weight,
   // which the decode right before it writes, so it waits first.
   constexpr bool kEarlyB = kKind == kKindI8;
+  // debug build: the skipped-stage fault leaves the first tile's stage 0
+  // empty in both CTAs (no expected bytes, no copies), so the MMA issuer's
+  // bounded wait on it runs out and the kernel takes its abort path
+  const bool skip0 = CONVROT_DEBUG && p.fault == kFaultSkipStage;
   int early = 0;  // stages of the first tile whose B load is already issued
   if (kEarlyB && threadIdx.x == 0 && unit < num_tiles) {
     int mb, nb;
@@ -241,6 +246,7 @@ __device__ __forceinline__ void gemm_pair(const CUtensorMap& tmA, const CUtensor
     const int b_row = nb * BN + static_cast<int>(rank) * C::kBRows;
     early = p.num_kb < C::kStages ? p.num_kb : C::kStages;
     for (int kb = 0; kb < early; ++kb) {  // fresh ring: every stage is free
+      if (skip0 && kb == 0) continue;
       if (leader) ptx::mbar_arrive_expect_tx(&bars->full[kb], C::kTxBytes);
       ptx::tma_load_2d_pair(sB + kb * C::kBStage, &tmB, &bars->full[kb], kb * KC::kStageK, b_row);
     }
@@ -264,6 +270,7 @@ __device__ __forceinline__ void gemm_pair(const CUtensorMap& tmA, const CUtensor
       tile_coords(unit, p.m_tiles, p.n_tiles, p.group_m, mb, nb);
       const int a_row = mb * C::kTileM + static_cast<int>(rank) * BM;
       for (int kb = 0; kb < early; ++kb) {
+        if (skip0 && kb == 0) continue;
         ptx::tma_load_2d_pair(sA + kb * A_STAGE, &tmA, &bars->full[kb], kb * KC::kStageK, a_row);
       }
       last_stage = early - 1;
@@ -279,6 +286,13 @@ __device__ __forceinline__ void gemm_pair(const CUtensorMap& tmA, const CUtensor
         if (!wait_bounded(&bars->empty[stage], phase ^ 1u)) {
           record_timeout(abort_flag, p.status);
           break;
+        }
+        if (skip0 && tile == unit && kb == 0) {  // (a form without early loads)
+          if (++stage == C::kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+          continue;
         }
         if (leader) ptx::mbar_arrive_expect_tx(&bars->full[stage], C::kTxBytes);
         ptx::tma_load_2d_pair(sA + stage * A_STAGE, &tmA, &bars->full[stage], kb * KC::kStageK, a_row);
@@ -364,6 +378,9 @@ __device__ __forceinline__ void gemm_pair(const CUtensorMap& tmA, const CUtensor
       ptx::tc_fence_after();
       const int64_t m = static_cast<int64_t>(mb) * C::kTileM + rank * BM + row;
       const bool row_ok = m < p.M;
+      // debug build: the rows this kernel may write (one fewer under the
+      // short-rows fault)
+      const int64_t m_limit = CONVROT_DEBUG && p.fault == kFaultShortRows ? p.M - 1 : p.M;
       float scale = kKind == kKindI8 ? 0.f : 1.f;
       if (kKind == kKindI8 && !p.out_s32 && row_ok) {
         scale = p.s_tok[m] * (p.per_channel_scale ? 1.f : p.s_w[0]);
@@ -376,7 +393,7 @@ __device__ __forceinline__ void gemm_pair(const CUtensorMap& tmA, const CUtensor
         ptx::tmem_ld_wait();
         const int64_t n0 = static_cast<int64_t>(nb) * BN + c * 32;
         const int valid = n0 + 32 <= p.N ? 32 : (n0 + 16 <= p.N ? 16 : 0);
-        if (row_ok && valid) {
+        if (row_ok && valid && in_bounds(m < m_limit && n0 + valid <= p.N, p.status)) {
           if (kKind == kKindI8 && p.out_s32) {
             store_s32_row32(static_cast<int32_t*>(p.out) + m * p.N + n0, r, valid);
           } else {
@@ -488,6 +505,7 @@ cudaError_t launch_int8_gemm(const GemmArgs& a, cudaStream_t stream) {
   p.per_channel_scale = a.s_w_len > 1 ? 1 : 0;
   p.out_s32 = a.out_s32 ? 1 : 0;
   p.out_f16 = a.out_f16 ? 1 : 0;
+  p.fault = debug_fault();
   // few tokens: the weight-streaming swap-AB kernel; otherwise CTA pairs
   // (256-row tiles) once there is more than one 128-row block of tokens
   if (a.M <= BM) return launch_int8_gemm_skinny(a, stream);
@@ -510,6 +528,7 @@ cudaError_t launch_gemm16(const GemmArgs& a, cudaStream_t stream) {
   p.per_channel_scale = 0;
   p.out_s32 = 0;
   p.out_f16 = a.out_f16 ? 1 : 0;
+  p.fault = debug_fault();
   return launch_pair(a, p, stream);
 }
 

@@ -48,7 +48,8 @@ struct SkinnyParams {
   int per_channel_scale;
   int out_s32;
   int out_f16;  // y and bias fp16 (else bf16)
-  unsigned int* status;
+  unsigned int* status;  // bit 0: a wait ran out; bit 1: debug bounds
+  int fault;             // debug build: injected fault (kFaultSkipStage, kFaultShortRows)
 };
 
 template <int NT>
@@ -142,8 +143,12 @@ __global__ void __launch_bounds__(kThreads, SkinnyCfg<NT>::kTwoPerSm ? 2 : 1)
   // producer issues the weight loads of its first stages before waiting on
   // that kernel: they stream while it drains.  The tokens' codes come after.
   const int early = kb1 - kb0 < kStages ? (kb1 > kb0 ? kb1 - kb0 : 0) : kStages;
+  // debug build: the skipped-stage fault leaves stage 0 empty (no expected
+  // bytes, no copies), so the MMA issuer's bounded wait on it runs out
+  const bool skip0 = CONVROT_DEBUG && p.fault == kFaultSkipStage;
   if (threadIdx.x == 0) {
     for (int i = 0; i < early; ++i) {  // fresh ring: every stage is free
+      if (skip0 && i == 0) continue;
       ptx::mbar_arrive_expect_tx(&bars->full[i], C::kStageBytes);
       ptx::tma_load_2d(sA + i * C::kAStage, &tmW, &bars->full[i], (kb0 + i) * kBK, block * kRows);
     }
@@ -157,6 +162,7 @@ __global__ void __launch_bounds__(kThreads, SkinnyCfg<NT>::kTwoPerSm ? 2 : 1)
     // ------------------------------------------------------------ producer
     // the early stages' codes first (always, so every issued stage completes)
     for (int i = 0; i < early; ++i) {
+      if (skip0 && i == 0) continue;
       ptx::tma_load_2d(sB + i * C::kBStage, &tmX, &bars->full[i], (kb0 + i) * kBK, 0);
     }
     int stage = early == kStages ? 0 : early;
@@ -239,6 +245,9 @@ __global__ void __launch_bounds__(kThreads, SkinnyCfg<NT>::kTwoPerSm ? 2 : 1)
       // timeout nothing is stored (the status word reports it).
       asm volatile("bar.sync 1, 128;" ::: "memory");
       const bool drain = ready && !__any_sync(0xffffffffu, *abort_flag != 0);
+      // debug build: the tokens this kernel may write (one fewer under the
+      // short-rows fault)
+      const int64_t m_limit = CONVROT_DEBUG && p.fault == kFaultShortRows ? p.M - 1 : p.M;
       const int64_t n = static_cast<int64_t>(block) * kRows + row;
       const float sw = p.out_s32 ? 0.f : ep_sw[row];
       const float bn = p.out_s32 ? 0.f : ep_bias[row];
@@ -252,6 +261,7 @@ __global__ void __launch_bounds__(kThreads, SkinnyCfg<NT>::kTwoPerSm ? 2 : 1)
         for (int j = 0; j < 16; ++j) {
           const int64_t m = c0 + j;
           if (m >= p.M) break;
+          if (!in_bounds(m < m_limit && n < p.N, p.status)) continue;
           if (p.out_s32) {
             static_cast<int32_t*>(p.out)[m * p.N + n] = static_cast<int32_t>(r[j]);
           } else {
@@ -341,10 +351,12 @@ __global__ void __launch_bounds__(kThreads, SkinnyCfg<NT>::kTwoPerSm ? 2 : 1)
       if (n >= p.N) continue;
       const float sw = p.out_s32 ? 0.f : ep_sw[r];
       const float bn = p.out_s32 ? 0.f : ep_bias[r];
+      const int64_t m_limit = CONVROT_DEBUG && p.fault == kFaultShortRows ? p.M - 1 : p.M;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int64_t m = m4 + j;
         if (m >= p.M) break;
+        if (!in_bounds(m < m_limit, p.status)) continue;
         if (p.out_s32) {
           static_cast<int32_t*>(p.out)[m * p.N + n] = a4[j];
         } else {
@@ -427,6 +439,7 @@ cudaError_t launch_int8_gemm_skinny(const GemmArgs& a, cudaStream_t stream) {
   p.per_channel_scale = a.s_w_len > 1 ? 1 : 0;
   p.out_s32 = a.out_s32 ? 1 : 0;
   p.out_f16 = a.out_f16 ? 1 : 0;
+  p.fault = debug_fault();
   if (a.M <= 16) return launch_nt<16>(a, p, stream);
   if (a.M <= 32) return launch_nt<32>(a, p, stream);
   if (a.M <= 64) return launch_nt<64>(a, p, stream);

@@ -15,7 +15,44 @@ struct convrot_rotation_s {
   float* Rt_dev;      // R transposed
 };
 
+// CONVROT_DEBUG=1 builds the debug library (libconvrot_debug.so): every
+// kernel checks the indices of its global stores and scale/bias reads
+// against the tensors' sizes, records a violation in bit 1 of the device
+// status word (convrot_check_status: CONVROT_ERR_BOUNDS) and skips the access
+// instead of trapping; and the host can inject faults for the tests
+// (convrot_debug_set_fault).  The release library compiles all of it out.
+#ifndef CONVROT_DEBUG
+#define CONVROT_DEBUG 0
+#endif
+
 namespace convrot {
+
+// Device status word bits.
+constexpr unsigned int kStatusTimeout = 1u;  // a bounded wait ran out
+constexpr unsigned int kStatusBounds = 2u;   // debug build: an index was out of range
+
+// Faults the debug library's tests inject from the host (0 = none).  The
+// launchers pass the current code to their kernels; the release library never
+// sets it.
+enum DebugFault : int {
+  kFaultNone = 0,
+  kFaultSkipStage = 1,   // int8 GEMM producers skip their first ring stage
+  kFaultShortRows = 2,   // kernels check stores against one token / row fewer
+};
+int debug_fault();
+void set_debug_fault(int code);
+
+// In the debug build: false (and bit 1 of the status word set) when `ok` is
+// false; the caller skips the access.  In the release build always true.
+__device__ __forceinline__ bool in_bounds(bool ok, unsigned int* status) {
+#if CONVROT_DEBUG
+  if (!ok) atomicOr(status, kStatusBounds);
+  return ok;
+#else
+  (void)status;
+  return true;
+#endif
+}
 
 // ------------------------------------------------------------------ rotations
 // Each launcher enqueues on `stream` and returns the launch error (cudaSuccess

@@ -490,7 +490,8 @@ __device__ __forceinline__ void unstage_chunk(uint32_t src, uint4 (&v)[kParts]) 
 template <int G, int kMaxThreads, int kMinBlocks, bool kF16>
 __global__ void __launch_bounds__(kMaxThreads, kMinBlocks) rotate_quant_act_hadamard(
     const uint16_t* __restrict__ x, int64_t M, int K, int team_warps, int rows_per_cta,
-    int8_t* __restrict__ xq, float* __restrict__ s_tok) {
+    int8_t* __restrict__ xq, float* __restrict__ s_tok, unsigned int* __restrict__ status,
+    int fault) {
   extern __shared__ __align__(16) uint8_t smem_all[];
   __shared__ float red[2][32];
   const int warp = threadIdx.x >> 5;
@@ -544,6 +545,9 @@ __global__ void __launch_bounds__(kMaxThreads, kMinBlocks) rotate_quant_act_hada
       amax = warp_max(static_cast<int>(lane) < team_warps ? rb_red[team * team_warps + lane] : 0.f);
     }
     if (!ok) continue;
+    // debug build: the token's codes and scale must lie inside xq and s_tok
+    const int64_t row_limit = CONVROT_DEBUG && fault == kFaultShortRows ? M - 1 : M;
+    if (!in_bounds(row < row_limit && (t + 1) * kVec <= K, status)) continue;
     const float sc = (amax * norm) / 127.f;  // s_tok = max |x_rot| / 127
     if (t == 0) s_tok[row] = sc;
     const float mul = norm * (sc > 0.f ? 1.f / sc : 0.f);  // exact scaling: norm is a power of two
@@ -575,7 +579,8 @@ __global__ void __launch_bounds__(256, MODE == kFlatDequant ? 3 : 4) hadamard_fl
                                                      uint64_t row_mul, int row_shift,
                                                      const float* __restrict__ scale,
                                                      void* __restrict__ out,
-                                                     unsigned int* __restrict__ absmax_bits) {
+                                                     unsigned int* __restrict__ absmax_bits,
+                                                     unsigned int* __restrict__ status, int fault) {
   constexpr int kParts = MODE == kFlatDequant ? 2 : 4;  // 16-byte parts of a chunk
   extern __shared__ __align__(16) uint8_t smem_all[];
   const uint32_t lane = threadIdx.x & 31;
@@ -598,6 +603,10 @@ __global__ void __launch_bounds__(256, MODE == kFlatDequant ? 3 : 4) hadamard_fl
   // the next block's chunks are copied into shared memory while this one is
   // transformed.  Lanes past the end copy nothing and transform stale data
   // (whole groups share `ok`); their results are dropped.
+  // debug build: the chunks this kernel may write (the last 256 elements,
+  // 8 chunks, fewer under the short-rows fault).  At G = 256 a lane's stores
+  // cover its whole group of 8 chunks, so its check covers the group.
+  const int64_t chunk_limit = CONVROT_DEBUG && fault == kFaultShortRows ? nchunks - 8 : nchunks;
   auto stage = [&](int64_t b) {
     const int64_t lim = lim0 - b * blockDim.x;
     stage_copies<kParts>(cp_dst, src + b * block_bytes,
@@ -633,7 +642,7 @@ __global__ void __launch_bounds__(256, MODE == kFlatDequant ? 3 : 4) hadamard_fl
     if constexpr (MODE == kFlatAbsmax) {
       if (ok) run_max = fmaxf(run_max, absmax32(P));
     } else if constexpr (MODE == kFlatQuant) {
-      if (ok) {
+      if (ok && in_bounds((G == 256 ? (c | 7) : c) < chunk_limit, status)) {
         int8_t* dst = static_cast<int8_t*>(out) + c * kVec;
         if (mul <= 3.0e38f) {
           store_codes32<G>(dst, P, mul, lane);
@@ -645,10 +654,11 @@ __global__ void __launch_bounds__(256, MODE == kFlatDequant ? 3 : 4) hadamard_fl
       // output row of chunk c: c / (K / 32) as a multiply and shift (row_reciprocal)
       const float sw =
           PER_ROW_SCALE ? scale[((ok ? static_cast<uint64_t>(c) : 0ull) * row_mul) >> row_shift] : scale[0];
+      const bool store_ok = in_bounds(!ok || (G == 256 ? (c | 7) : c) < chunk_limit, status);
       uint32_t w[kPairs];
       products16_32<kF16>(w, P, sw * norm);
       if constexpr (G == 256) {
-        if (ok) store_words16<G>(static_cast<uint16_t*>(out) + c * kVec, w, lane);
+        if (ok && store_ok) store_words16<G>(static_cast<uint16_t*>(out) + c * kVec, w, lane);
       } else {
         // A lane's 64 output bytes are 4 units of the warp's 2 KB; through the
         // output slot, store j of lane i writes unit 32 j + i (512 contiguous
@@ -667,7 +677,7 @@ __global__ void __launch_bounds__(256, MODE == kFlatDequant ? 3 : 4) hadamard_fl
         const uint32_t rd = aux + stage_copy_offset(lane);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          if (8 * j < olim) {
+          if (8 * j < olim && in_bounds(chunk0 + 8 * j + static_cast<int>(lane >> 2) < chunk_limit, status)) {
             uint4 v;
             asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
                          : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
@@ -864,8 +874,11 @@ cudaError_t rqa_launch(const uint16_t* x, int64_t M, int K, int team_warps, int 
   const int64_t blocks = (M + rows_per_cta - 1) / rows_per_cta;
   const int64_t cap = static_cast<int64_t>(sm_count()) * (per_sm > 0 ? per_sm : 1);
   const int64_t grid = blocks < cap ? blocks : cap;
+  unsigned int* status = nullptr;
+  e = status_word(&status);
+  if (e != cudaSuccess) return e;
   return launch_chained(rotate_quant_act_hadamard<G, kMaxThreads, kMinBlocks, kF16>, grid, 32 * warps, smem,
-                        stream, x, M, K, team_warps, rows_per_cta, xq, s_tok);
+                        stream, x, M, K, team_warps, rows_per_cta, xq, s_tok, status, debug_fault());
 }
 
 template <int G, bool kF16>
@@ -925,8 +938,11 @@ cudaError_t flat_launch(const void* in, int64_t nchunks, int64_t chunks_per_row,
     if (nchunks >= (1ll << 31) || chunks_per_row < 1) return cudaErrorInvalidValue;
     row_reciprocal(static_cast<uint64_t>(chunks_per_row), &row_mul, &row_shift);
   }
+  unsigned int* status = nullptr;
+  e = status_word(&status);
+  if (e != cudaSuccess) return e;
   return launch_chained(hadamard_flat<G, MODE, PER_ROW, kF16>, grid, kThreadsFlat, smem, stream, in,
-                        nchunks, row_mul, row_shift, scale, out, absmax_bits);
+                        nchunks, row_mul, row_shift, scale, out, absmax_bits, status, debug_fault());
 }
 
 template <int G, typename TIn, int MODE, bool kF16>

@@ -53,7 +53,9 @@ typedef enum convrot_status {
   CONVROT_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed */
   CONVROT_ERR_WORKSPACE = 4,    /* workspace missing or smaller than convrot_workspace_bytes() */
   CONVROT_ERR_TIMEOUT = 5,      /* a bounded wait inside a kernel ran out */
-  CONVROT_ERR_ALIGNMENT = 6     /* a pointer is not 16-byte aligned */
+  CONVROT_ERR_ALIGNMENT = 6,    /* a pointer is not 16-byte aligned */
+  CONVROT_ERR_BOUNDS = 7        /* debug library only (convrot_debug.h): a kernel caught an
+                                   out-of-range index and skipped that access */
 } convrot_status;
 
 typedef uint16_t convrot_bf16;                     /* bfloat16 bit pattern */
@@ -331,7 +333,9 @@ size_t convrot_workspace_bytes(int op, int64_t M, int64_t N, int64_t K);
 /*
  * Synchronizes `stream`, then reads and clears the current device's status
  * word: CONVROT_ERR_TIMEOUT if a kernel gave up a wait since the last check,
- * CONVROT_ERR_CUDA if the synchronization reported an error, else CONVROT_OK.
+ * CONVROT_ERR_BOUNDS if (debug library only) a kernel caught an out-of-range
+ * index, CONVROT_ERR_CUDA if the synchronization reported an error, else
+ * CONVROT_OK.
  */
 convrot_status convrot_check_status(convrot_stream_t stream);
 

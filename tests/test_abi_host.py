@@ -24,8 +24,11 @@ FAKE = 0x10000          # a 16-byte aligned address that is never dereferenced
 MISALIGNED = 0x10008
 
 
-def declared_functions():
-    text = open(HEADER).read()
+DEBUG_HEADER = os.path.join(ROOT, "include", "convrot_debug.h")
+
+
+def declared_functions(header=HEADER):
+    text = open(header).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
     return sorted(set(re.findall(r"\b(convrot_[a-z0-9_]+)\s*\(", text)))
 
@@ -197,3 +200,24 @@ def test_header_compiles_as_c_and_links(tmp_path):
     res = subprocess.run([exe], capture_output=True, text=True, timeout=120)
     assert res.returncode == 0, res.stderr
     assert "c abi ok" in res.stdout
+
+
+def test_debug_library_exports_both_headers():
+    """libconvrot_debug.so (CONVROT_DEBUG=1) exports everything convrot.h
+    declares plus the fault hook of convrot_debug.h; the release library
+    does not export the hook."""
+    dbg = ctypes.CDLL(build.DEBUG_LIB_PATH)
+    for n in declared_functions() + declared_functions(DEBUG_HEADER):
+        assert hasattr(dbg, n), f"{n} not exported by the debug library"
+    assert declared_functions(DEBUG_HEADER) == ["convrot_debug_set_fault"]
+    assert not hasattr(ctypes.CDLL(build.LIB_PATH), "convrot_debug_set_fault")
+
+
+def test_debug_fault_codes_checked_on_the_host():
+    dbg = cr.load_library(build.DEBUG_LIB_PATH)
+    f = dbg.convrot_debug_set_fault
+    f.argtypes = [ctypes.c_int]
+    f.restype = ctypes.c_int
+    assert f(3) == cr.INVALID_ARG and f(-1) == cr.INVALID_ARG
+    assert b"unknown fault" in dbg.convrot_last_error_string()
+    assert f(0) == cr.OK
