@@ -400,7 +400,10 @@ cudaError_t launch_nt(const GemmArgs& a, SkinnyParams p, cudaStream_t stream) {
                                        static_cast<int>(C::kSmem));
   if (e != cudaSuccess) return e;
   const int blocks = static_cast<int>((a.N + kRows - 1) / kRows);
-  int splits = sm_count() / blocks;  // one CTA per SM, one wave
+  // as many CTAs as fit in one wave: two per SM when the ring is sized for it
+  // (chained few-token launches over 3840 x 11520 and 10240 x 3840 weights
+  // measured 6 and 10 % faster than with one CTA per SM's worth of splits)
+  int splits = (C::kTwoPerSm ? 2 : 1) * sm_count() / blocks;
   splits = splits < 1 ? 1 : (splits > 8 ? 8 : splits);
   if (splits > p.num_kb) splits = p.num_kb;
   while (kRows % splits) --splits;  // each rank finishes an equal share of the 128 rows
