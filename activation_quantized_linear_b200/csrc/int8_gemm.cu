@@ -65,7 +65,10 @@ struct Cfg {
   static constexpr int kStageBytes = A_STAGE + kBStage;
   static constexpr int kStages = 6;
   static constexpr int kTileM = 2 * BM;
-  static constexpr size_t kSmem = 1024 + kStages * kStageBytes + 256;
+  // each epilogue warp's copy of a tile's 256 bias values and 256 weight
+  // scales (float)
+  static constexpr int kEpiWarpBytes = 2 * BN * 4;
+  static constexpr size_t kSmem = 1024 + kStages * kStageBytes + 256 + 4 * kEpiWarpBytes;
   // bytes that complete one stage on the leader's full barrier (both CTAs' loads)
   static constexpr uint32_t kTxBytes = 2 * kStageBytes;
 };
@@ -135,28 +138,27 @@ __device__ __forceinline__ float widen16(uint16_t v, bool f16) {
   return f16 ? __half2float(__ushort_as_half(v)) : __uint_as_float(static_cast<uint32_t>(v) << 16);
 }
 
-// `valid` (16 or 32) of the 32 columns exist.  Columns 16..31 read their
-// scale and bias through a second base that falls back to columns 0..15 when
-// only 16 exist, so nothing past N is read (those outputs are not stored).
+// 32 outputs of one row: y = f16(float(acc) * scale [* s_w[col]] + bias[col]),
+// in bf16 or fp16 (f16), rounded once from the fp32 FMA, with the tile's bias
+// and weight scales read from the warp's shared-memory copy (float; `bias`
+// null: none, `s_w` null: per tensor).  The accumulator columns hold int32
+// (kF32Acc = false) or fp32 (true: scale is 1, so y = f16(acc + bias)).
+// `valid` (16 or 32) of the 32 columns exist.
 template <bool kF32Acc>
-__device__ __forceinline__ void store_row32(uint16_t* dst, const uint32_t (&r)[32], float scale,
-                                            const float* s_w_row, const uint16_t* bias, int valid,
-                                            bool f16) {
-  const int hi_base = valid == 32 ? 16 : 0;
+__device__ __forceinline__ void store_row32_staged(uint16_t* dst, const uint32_t (&r)[32], float scale,
+                                                   const float* s_w, const float* bias, int valid,
+                                                   bool f16) {
   uint32_t w[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
-    const int col = i < 8 ? 2 * i : 2 * i - 16 + hi_base;
+    // columns past a half-filled chunk read staged zeros and are not stored
+    const int col = 2 * i;
     float lo = kF32Acc ? __uint_as_float(r[2 * i]) : __int2float_rn(static_cast<int32_t>(r[2 * i]));
     float hi = kF32Acc ? __uint_as_float(r[2 * i + 1])
                        : __int2float_rn(static_cast<int32_t>(r[2 * i + 1]));
-    const float sl = s_w_row ? scale * s_w_row[col] : scale;
-    const float sh = s_w_row ? scale * s_w_row[col + 1] : scale;
-    float bl = 0.f, bh = 0.f;
-    if (bias) {
-      bl = widen16(bias[col], f16);
-      bh = widen16(bias[col + 1], f16);
-    }
+    const float sl = s_w ? scale * s_w[col] : scale;
+    const float sh = s_w ? scale * s_w[col + 1] : scale;
+    const float bl = bias ? bias[col] : 0.f, bh = bias ? bias[col + 1] : 0.f;
     lo = fmaf(lo, sl, bl);
     hi = fmaf(hi, sh, bh);
     if (f16) {
@@ -195,6 +197,8 @@ __device__ __forceinline__ void gemm_pair(const CUtensorMap& tmA, const CUtensor
   uint8_t* sA = smem;
   uint8_t* sB = smem + C::kStages * A_STAGE;
   auto* bars = reinterpret_cast<Barriers<C::kStages>*>(smem + C::kStages * C::kStageBytes);
+  static_assert(sizeof(Barriers<C::kStages>) <= 256, "barriers must fit their 256 bytes");
+  float* ep_all = reinterpret_cast<float*>(smem + C::kStages * C::kStageBytes + 256);
   volatile uint32_t* abort_flag = &bars->abort_flag;
 
   const int warp = threadIdx.x >> 5;
@@ -364,12 +368,53 @@ __device__ __forceinline__ void gemm_pair(const CUtensorMap& tmA, const CUtensor
     // ------------------------------------------------------------ epilogue
     const int quarter = warp & 3;  // TMEM lanes this warp may read: 32*quarter ..
     const int row = quarter * 32 + static_cast<int>(lane);
+    // this warp's copy of the tile's factors: bias [BN], weight scales [BN]
+    float* ep_bias = ep_all + (warp - 2) * (C::kEpiWarpBytes / 4);
+    float* ep_sw = ep_bias + BN;
+    const bool has_bias = p.bias != nullptr;
+    const bool chan_sw = kKind == kKindI8 && p.per_channel_scale && !p.out_s32;
     int local = 0;
     for (int tile = unit; tile < num_tiles; tile += units, ++local) {
       int mb, nb;
       tile_coords(tile, p.m_tiles, p.n_tiles, p.group_m, mb, nb);
       const int acc = local & 1;
       const uint32_t acc_phase = (local >> 1) & 1;
+      // Stage the tile's bias and per-channel scales before waiting for its
+      // accumulator, so the loads overlap the tile's MMAs instead of
+      // following each 32-column chunk: lane i takes columns 8i .. 8i + 7
+      // (N % 16 == 0, so such a group is wholly inside or outside N).
+      __syncwarp();  // the previous tile's copy is no longer read
+      {
+        const int64_t col = static_cast<int64_t>(nb) * BN + 8 * lane;
+        const bool in_n = col < p.N;
+        float b8[8], s8[8];
+        if (has_bias && in_n) {
+          const uint4 v = *reinterpret_cast<const uint4*>(p.bias + col);
+          const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            b8[2 * k] = widen16(static_cast<uint16_t>(wv[k] & 0xffffu), p.out_f16 != 0);
+            b8[2 * k + 1] = widen16(static_cast<uint16_t>(wv[k] >> 16), p.out_f16 != 0);
+          }
+        } else {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) b8[k] = 0.f;
+        }
+        if (chan_sw && in_n) {
+          const float4 a = *reinterpret_cast<const float4*>(p.s_w + col);
+          const float4 b = *reinterpret_cast<const float4*>(p.s_w + col + 4);
+          s8[0] = a.x; s8[1] = a.y; s8[2] = a.z; s8[3] = a.w;
+          s8[4] = b.x; s8[5] = b.y; s8[6] = b.z; s8[7] = b.w;
+        } else {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) s8[k] = 0.f;
+        }
+        *reinterpret_cast<float4*>(ep_bias + 8 * lane) = make_float4(b8[0], b8[1], b8[2], b8[3]);
+        *reinterpret_cast<float4*>(ep_bias + 8 * lane + 4) = make_float4(b8[4], b8[5], b8[6], b8[7]);
+        *reinterpret_cast<float4*>(ep_sw + 8 * lane) = make_float4(s8[0], s8[1], s8[2], s8[3]);
+        *reinterpret_cast<float4*>(ep_sw + 8 * lane + 4) = make_float4(s8[4], s8[5], s8[6], s8[7]);
+      }
+      __syncwarp();
       const bool ready = __all_sync(0xffffffffu, wait_bounded(&bars->acc_full[acc], acc_phase));
       if (!ready) {
         if (lane == 0) record_timeout(abort_flag, p.status);
@@ -397,10 +442,10 @@ __device__ __forceinline__ void gemm_pair(const CUtensorMap& tmA, const CUtensor
           if (kKind == kKindI8 && p.out_s32) {
             store_s32_row32(static_cast<int32_t*>(p.out) + m * p.N + n0, r, valid);
           } else {
-            store_row32<kKind != kKindI8>(
-                static_cast<uint16_t*>(p.out) + m * p.N + n0, r, scale,
-                kKind == kKindI8 && p.per_channel_scale ? p.s_w + n0 : nullptr,
-                p.bias ? p.bias + n0 : nullptr, valid, p.out_f16 != 0);
+            store_row32_staged<kKind != kKindI8>(static_cast<uint16_t*>(p.out) + m * p.N + n0, r,
+                                                 scale, chan_sw ? ep_sw + c * 32 : nullptr,
+                                                 has_bias ? ep_bias + c * 32 : nullptr, valid,
+                                                 p.out_f16 != 0);
           }
         }
       }

@@ -515,6 +515,23 @@ def run_sweep(args):
                          "gemm_frac_int8_peak": ops / t_g / 1e9 / int8_peak,
                          "gemm_GBps": gemm_bytes / t_g / 1e6,
                          "gemm_frac_hbm": gemm_bytes / t_g / 1e6 / hbm_gbs})
+    # GEMMs launched back to back as in use (chained: each launch's set-up and
+    # first weight loads overlap the previous launch's drain), each on its own
+    # weight copy so that the weights stream from HBM; K = N = 4096
+    gemm_chained = []
+    rot = cr.Rotation(workloads.sylvester_rotation(256))
+    for Mc in (1024, 8192):
+        Ws = [torch.randint(-127, 128, (4096, 4096), dtype=torch.int8, device="cuda") for _ in range(6)]
+        xq = torch.randint(-127, 128, (Mc, 4096), dtype=torch.int8, device="cuda")
+        st = torch.rand(Mc, device="cuda") * 1e-3
+        sw1 = torch.tensor([1e-3], device="cuda")
+        bias = torch.zeros(4096, dtype=torch.bfloat16, device="cuda")
+        y = torch.empty((Mc, 4096), dtype=torch.bfloat16, device="cuda")
+        t = timed(lambda: [cr.int8_gemm(xq, st, W, sw1, bias, out=y) for W in Ws], args.steps) / len(Ws)
+        ops = 2.0 * Mc * 4096 * 4096
+        gemm_chained.append({"M": Mc, "gemm_ms": t, "gemm_TOPS": ops / t / 1e9,
+                             "gemm_frac_int8_peak": ops / t / 1e9 / int8_peak})
+        del Ws
     dec = []
     N, K = workloads.DEROTATE_SWEEP_SHAPE
     for G in workloads.GROUP_SIZES:
@@ -588,6 +605,7 @@ def run_sweep(args):
                       "decode_12288x3072_ms": t_d, "decode_GBps": 3 * N * K / t_d / 1e6,
                       "decode_fp64_tflops": 2.0 * G * N * K / t_d / 1e9})
     print(json.dumps({"sweep": "group_size_and_skinny_M", "linears": rows, "decode_12288x3072": dec,
+                      "gemm_chained_K4096": gemm_chained,
                       "variants_G256": var, "dense_R_M8192": dense,
                       "few_tokens_chained_G256": chained,
                       "peaks": {"hbm_gbs": hbm_gbs, "int8_tops": int8_peak}}))

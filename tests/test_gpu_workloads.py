@@ -136,9 +136,11 @@ def test_decode_12288x3072(cr, G):
 # part of the CTA-pair GEMM's schedule: the Z-Image QKV (36 x 45 tiles, several
 # persistent passes per pair, s32 output wider than 1024 columns), the Wan
 # down-projection (M*K > 64 MB: the grouped tile raster), K = N = 4096 at
-# M = 8192 (512 tiles: many waves of the double-buffered TMEM accumulators).
+# M = 8192 (512 tiles: many waves of the double-buffered TMEM accumulators),
+# K = N = 4096 at M = 1024 (64 tiles on the 74 CTA pairs: one wave).
 S32_FULL = [("zimage_qkv", 4608, 11520, 3840), ("wan_down", 7800, 5120, 13824),
-            ("k4096_m8192", 8192, 4096, 4096), ("flux_in_proj", 4608, 21504, 3072)]
+            ("k4096_m8192", 8192, 4096, 4096), ("flux_in_proj", 4608, 21504, 3072),
+            ("k4096_m1024_one_wave", 1024, 4096, 4096)]
 
 
 @pytest.mark.parametrize("name,M,N,K", S32_FULL, ids=[c[0] for c in S32_FULL])
