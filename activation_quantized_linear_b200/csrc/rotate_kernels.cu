@@ -484,10 +484,37 @@ __device__ __forceinline__ void unstage_chunk(uint32_t src, uint4 (&v)[kParts]) 
   }
 }
 
+// The named barrier of team `team` (ID 1 + team) for the kTeams teams of a
+// CTA, its ID an immediate: ptxas then reserves only those IDs, where a
+// register-valued ID reserves all 16 of the CTA, and the occupancy
+// calculation admitted only 4 CTAs of 5 warps per SM although registers and
+// shared memory allow 5.  kTeams == 0: one-warp teams, no barrier.
+template <int kTeams>
+__device__ __forceinline__ void team_barrier(int team, int nthreads) {
+  static_assert(kTeams == 0 || kTeams == 1 || kTeams == 2 || kTeams == 4, "teams per CTA");
+  if constexpr (kTeams == 1) {
+    asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
+  } else if constexpr (kTeams == 2) {
+    if (team == 0) {
+      asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
+    } else {
+      asm volatile("bar.sync 2, %0;" ::"r"(nthreads) : "memory");
+    }
+  } else if constexpr (kTeams == 4) {
+    switch (team) {
+      case 0: asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory"); break;
+      case 1: asm volatile("bar.sync 2, %0;" ::"r"(nthreads) : "memory"); break;
+      case 2: asm volatile("bar.sync 3, %0;" ::"r"(nthreads) : "memory"); break;
+      default: asm volatile("bar.sync 4, %0;" ::"r"(nthreads) : "memory"); break;
+    }
+  }
+}
+
 // Register budgets by CTA size: kMaxThreads threads, kMinBlocks CTAs per SM
 // (256, 3) and (384, 2) leave room for 85 registers; (1024, 1) keeps 64, so
-// that teams of up to 512 threads still fit two CTAs per SM.
-template <int G, int kMaxThreads, int kMinBlocks, bool kF16>
+// that teams of up to 512 threads still fit two CTAs per SM.  kTeams: teams
+// (token rows) per CTA, 0 for one-warp teams.
+template <int G, int kMaxThreads, int kMinBlocks, bool kF16, int kTeams>
 __global__ void __launch_bounds__(kMaxThreads, kMinBlocks) rotate_quant_act_hadamard(
     const uint16_t* __restrict__ x, int64_t M, int K, int team_warps, int rows_per_cta,
     int8_t* __restrict__ xq, float* __restrict__ s_tok, unsigned int* __restrict__ status,
@@ -515,7 +542,7 @@ __global__ void __launch_bounds__(kMaxThreads, kMinBlocks) rotate_quant_act_hada
   // block's chunks are copied into shared memory while this one is transformed.
   // Lanes without a chunk (the row's tail, rows past M) copy nothing and
   // transform stale data; whole groups share `ok`, and their results are dropped.
-  const int bar_id = 1 + team, bar_threads = team_warps * 32;
+  const int bar_threads = team_warps * 32;
   const int64_t row_step = static_cast<int64_t>(gridDim.x) * rows_per_cta;
   // launched chained to the previous kernel: global memory only after it completes
   ptx::grid_dependency_wait();
@@ -537,11 +564,11 @@ __global__ void __launch_bounds__(kMaxThreads, kMinBlocks) rotate_quant_act_hada
     stage_copies<4>(cp_dst, src, row + row_step < M ? lim : 0);
     fwht32<G, false>(P, xch, lane);
     float amax = warp_max(ok ? absmax32(P) : 0.f);
-    if (team_warps > 1) {
+    if (kTeams > 0) {
       float* rb_red = red[it & 1];
       if (lane == 0) rb_red[warp] = amax;
       // the team's warps only: teams of one CTA run independently
-      asm volatile("bar.sync %0, %1;" ::"r"(bar_id), "r"(bar_threads) : "memory");
+      team_barrier<kTeams>(team, bar_threads);
       amax = warp_max(static_cast<int>(lane) < team_warps ? rb_red[team * team_warps + lane] : 0.f);
     }
     if (!ok) continue;
@@ -858,17 +885,17 @@ cudaError_t allow_smem(Kern kern, size_t bytes) {
                               static_cast<int>(bytes));
 }
 
-template <int G, int kMaxThreads, int kMinBlocks, bool kF16>
+template <int G, int kMaxThreads, int kMinBlocks, bool kF16, int kTeams>
 cudaError_t rqa_launch(const uint16_t* x, int64_t M, int K, int team_warps, int rows_per_cta,
                        int8_t* xq, float* s_tok, cudaStream_t stream) {
   const int warps = team_warps * rows_per_cta;
   const size_t smem = static_cast<size_t>(warps) * (kStageBytesPerWarp + xch_bytes_per_warp<G>());
-  cudaError_t e = allow_smem(rotate_quant_act_hadamard<G, kMaxThreads, kMinBlocks, kF16>, smem);
+  cudaError_t e = allow_smem(rotate_quant_act_hadamard<G, kMaxThreads, kMinBlocks, kF16, kTeams>, smem);
   if (e != cudaSuccess) return e;
   // enough CTAs to fill every SM (register-limited occupancy), each looping
   // over row blocks with a one-block-ahead prefetch
   int per_sm = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, rotate_quant_act_hadamard<G, kMaxThreads, kMinBlocks, kF16>,
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, rotate_quant_act_hadamard<G, kMaxThreads, kMinBlocks, kF16, kTeams>,
                                                     32 * warps, smem);
   if (e != cudaSuccess) return e;
   const int64_t blocks = (M + rows_per_cta - 1) / rows_per_cta;
@@ -877,7 +904,7 @@ cudaError_t rqa_launch(const uint16_t* x, int64_t M, int K, int team_warps, int 
   unsigned int* status = nullptr;
   e = status_word(&status);
   if (e != cudaSuccess) return e;
-  return launch_chained(rotate_quant_act_hadamard<G, kMaxThreads, kMinBlocks, kF16>, grid, 32 * warps, smem,
+  return launch_chained(rotate_quant_act_hadamard<G, kMaxThreads, kMinBlocks, kF16, kTeams>, grid, 32 * warps, smem,
                         stream, x, M, K, team_warps, rows_per_cta, xq, s_tok, status, debug_fault());
 }
 
@@ -893,13 +920,24 @@ cudaError_t rqa_hadamard(const uint16_t* x, int64_t M, int64_t K, int8_t* xq, fl
   const int k = static_cast<int>(K);
   // 9-10 warps fit three CTAs per SM only at 64 registers; 11-12 fit two
   // CTAs either way, so they take the larger budget
+  // teams per CTA: 8 one-warp teams (no barrier), 4 of 2 warps, 2 of 3-4,
+  // else 1
   if (warps <= 8) {
-    return rqa_launch<G, 256, 3, kF16>(x, M, k, team_warps, rows_per_cta, xq, s_tok, stream);
+    if (team_warps == 1) {
+      return rqa_launch<G, 256, 3, kF16, 0>(x, M, k, team_warps, rows_per_cta, xq, s_tok, stream);
+    }
+    if (rows_per_cta == 4) {
+      return rqa_launch<G, 256, 3, kF16, 4>(x, M, k, team_warps, rows_per_cta, xq, s_tok, stream);
+    }
+    if (rows_per_cta == 2) {
+      return rqa_launch<G, 256, 3, kF16, 2>(x, M, k, team_warps, rows_per_cta, xq, s_tok, stream);
+    }
+    return rqa_launch<G, 256, 3, kF16, 1>(x, M, k, team_warps, rows_per_cta, xq, s_tok, stream);
   }
   if (warps >= 11 && warps <= 12) {
-    return rqa_launch<G, 384, 2, kF16>(x, M, k, team_warps, rows_per_cta, xq, s_tok, stream);
+    return rqa_launch<G, 384, 2, kF16, 1>(x, M, k, team_warps, rows_per_cta, xq, s_tok, stream);
   }
-  return rqa_launch<G, 1024, 1, kF16>(x, M, k, team_warps, rows_per_cta, xq, s_tok, stream);
+  return rqa_launch<G, 1024, 1, kF16, 1>(x, M, k, team_warps, rows_per_cta, xq, s_tok, stream);
 }
 
 // Multiplier m and shift k with floor(c * m / 2^k) == c / d for every
