@@ -171,18 +171,28 @@ __device__ __forceinline__ void widen_stage0_32(const uint4 (&u)[4], uint64_t (&
   }
 }
 
-// raw int8 words -> P[i] = (p[2i], p[2i + 1]) as floats.
-__device__ __forceinline__ void widen_i8_32(const uint4 (&u)[2], uint64_t (&P)[kPairs]) {
+// raw int8 words -> P after butterfly bits 0 and 1: each word holds four
+// elements b0..b3, and dp4a against the +-1 sign words of the 4-point
+// transform gives its four outputs as exact integers (|y| <= 508).  The
+// accumulator 0x4B400000 is 1.5 * 2^23 as a float, so each result read as a
+// float is 1.5 * 2^23 + y exactly; one packed subtraction leaves y.
+//   P[2k] = (b0 + b1 + b2 + b3, b0 - b1 + b2 - b3),
+//   P[2k + 1] = (b0 + b1 - b2 - b3, b0 - b1 - b2 + b3)   (word k).
+__device__ __forceinline__ void widen_i8_wht4_32(const uint4 (&u)[2], uint64_t (&P)[kPairs]) {
+  constexpr int kMagicBits = 0x4B400000;
+  const uint64_t magic2 = pk(kRoundMagic, kRoundMagic);
 #pragma unroll
   for (int j = 0; j < 2; ++j) {
     const int w[4] = {static_cast<int>(u[j].x), static_cast<int>(u[j].y),
                       static_cast<int>(u[j].z), static_cast<int>(u[j].w)};
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-      P[8 * j + 2 * k] = pk(static_cast<float>(static_cast<int8_t>(w[k])),
-                            static_cast<float>(static_cast<int8_t>(w[k] >> 8)));
-      P[8 * j + 2 * k + 1] = pk(static_cast<float>(static_cast<int8_t>(w[k] >> 16)),
-                                static_cast<float>(w[k] >> 24));
+      const int y0 = __dp4a(w[k], 0x01010101, kMagicBits);
+      const int y1 = __dp4a(w[k], static_cast<int>(0xFF01FF01u), kMagicBits);
+      const int y2 = __dp4a(w[k], static_cast<int>(0xFFFF0101u), kMagicBits);
+      const int y3 = __dp4a(w[k], static_cast<int>(0x01FFFF01u), kMagicBits);
+      P[8 * j + 2 * k] = sub2(pku(y0, y1), magic2);
+      P[8 * j + 2 * k + 1] = sub2(pku(y2, y3), magic2);
     }
   }
 }
@@ -204,10 +214,12 @@ __device__ __forceinline__ void widen_i8_32(const uint4 (&u)[2], uint64_t (&P)[k
 constexpr int kXchGroupBytes = 8 * 9 * 16 + 8;
 constexpr int kXchBytesPerWarp = 4 * kXchGroupBytes;  // 4 groups
 
-// kStage0 = false: bit 0 was already applied (widen_stage0_32).
-template <int G, bool kStage0 = true>
+// kDone: element bits already transformed by the widening (0; 1 after
+// widen_stage0_32; 2 after widen_i8_wht4_32).
+template <int G, int kDone>
 __device__ __forceinline__ void fwht32(uint64_t (&P)[kPairs], uint32_t xch, uint32_t lane) {
-  if constexpr (kStage0) {
+  static_assert(kDone >= 0 && kDone <= 2, "stages done by the widening");
+  if constexpr (kDone == 0) {
 #pragma unroll
     for (int i = 0; i < kPairs; ++i) {  // bit 0
       const float a = plo(P[i]), b = phi(P[i]);
@@ -216,7 +228,7 @@ __device__ __forceinline__ void fwht32(uint64_t (&P)[kPairs], uint32_t xch, uint
   }
   constexpr int kTop = (G < kVec ? G : kVec) / 2;  // pair-index stages (bits 1..)
 #pragma unroll
-  for (int h = 1; h < kTop; h <<= 1) {
+  for (int h = kDone == 2 ? 2 : 1; h < kTop; h <<= 1) {
 #pragma unroll
     for (int i = 0; i < kPairs; ++i) {
       if ((i & h) == 0) {
@@ -562,7 +574,7 @@ __global__ void __launch_bounds__(kMaxThreads, kMinBlocks) rotate_quant_act_hada
     __syncwarp();  // every lane has read its units before the slot is refilled
     src += src_step;
     stage_copies<4>(cp_dst, src, row + row_step < M ? lim : 0);
-    fwht32<G, false>(P, xch, lane);
+    fwht32<G, 1>(P, xch, lane);
     float amax = warp_max(ok ? absmax32(P) : 0.f);
     if (kTeams > 0) {
       float* rb_red = red[it & 1];
@@ -658,13 +670,17 @@ __global__ void __launch_bounds__(256, MODE == kFlatDequant ? 3 : 4) hadamard_fl
     unstage_chunk<kParts>(rd_src, u);
     uint64_t P[kPairs];
     if constexpr (MODE == kFlatDequant) {
-      widen_i8_32(u, P);
+      widen_i8_wht4_32(u, P);
     } else {
       widen16_32<kF16>(u, P);
     }
     __syncwarp();  // every lane has read its units before the slot is refilled
     stage(b + gridDim.x);
-    fwht32<G>(P, aux, lane);
+    if constexpr (MODE == kFlatDequant) {
+      fwht32<G, 2>(P, aux, lane);
+    } else {
+      fwht32<G, 0>(P, aux, lane);
+    }
 
     if constexpr (MODE == kFlatAbsmax) {
       if (ok) run_max = fmaxf(run_max, absmax32(P));
