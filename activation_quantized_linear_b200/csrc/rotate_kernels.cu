@@ -587,7 +587,14 @@ __global__ void __launch_bounds__(kMaxThreads, kMinBlocks) rotate_quant_act_hada
     // debug build: the token's codes and scale must lie inside xq and s_tok
     const int64_t row_limit = CONVROT_DEBUG && fault == kFaultShortRows ? M - 1 : M;
     if (!in_bounds(row < row_limit && (t + 1) * kVec <= K, status)) continue;
-    const float sc = (amax * norm) / 127.f;  // s_tok = max |x_rot| / 127
+    // s_tok = max |x_rot| / 127, correctly rounded without a division.  With
+    // a = amax * norm (exact) and m any float32 rounding midpoint of a / 127,
+    // a - 127 m is an odd multiple of half the quotient's ulp (a's bits are
+    // even multiples of it, 127 times an odd multiple is odd), so a / 127 lies
+    // at least 2^-31 (relative) from every midpoint, and 2^-150 / 127 away when
+    // the quotient is subnormal.  The float64 product a * RN(1/127) is within
+    // 2^-52 (relative) of a / 127, so its one rounding to float32 is RN(a / 127).
+    const float sc = static_cast<float>(static_cast<double>(amax * norm) * (1.0 / 127.0));
     if (t == 0) s_tok[row] = sc;
     const float mul = norm * (sc > 0.f ? 1.f / sc : 0.f);  // exact scaling: norm is a power of two
     int8_t* dst = xq + row * K + static_cast<int64_t>(t) * kVec;

@@ -171,6 +171,30 @@ def test_rotate_quant_act_parity(G, kind, M, K):
     assert float(s_tok[min(2, M - 1)]) == 0.0 and not xq[min(2, M - 1)].any()
 
 
+@pytest.mark.parametrize("G", [16, 256])
+def test_token_scale_is_the_correctly_rounded_quotient(G):
+    """s_tok = RN_float32(max|x_rot| / 127), bit for bit.  Token i holds one
+    nonzero element v_i, so its rotated row is +-v_i / sqrt(G) in one group
+    and the absmax |v_i| / sqrt(G) is exact; the expected scale is the float32
+    quotient, which numpy rounds once (float32 division is IEEE).  The v_i span
+    normal scales and the tiny ones whose scale is a float32 subnormal."""
+    rng = np.random.default_rng(77 + G)
+    M, K = 4096, 512
+    exps = np.concatenate([rng.uniform(-40.0, 60.0, M - 512), rng.uniform(-124.0, -112.0, 512)])
+    v = (rng.uniform(1.0, 2.0, M) * np.exp2(exps) * rng.choice([-1.0, 1.0], M))
+    v = torch.from_numpy(v).to(torch.bfloat16)
+    x = torch.zeros((M, K), dtype=torch.bfloat16)
+    cols = torch.from_numpy(rng.integers(0, K, M))
+    x[torch.arange(M), cols] = v
+    rot = cr.Rotation(workloads.sylvester_rotation(G))
+    _, s_tok = cr.rotate_quant_act(x.cuda(), rot)
+    a = (np.abs(v.float().numpy()) * np.float32(1.0 / np.sqrt(G))).astype(np.float32)
+    assert np.all(a > 0)
+    expect = a / np.float32(127.0)
+    assert np.any(expect < np.finfo(np.float32).tiny)  # subnormal scales are covered
+    np.testing.assert_array_equal(s_tok.cpu().numpy().view(np.uint32), expect.view(np.uint32))
+
+
 def test_rotate_quant_act_empty():
     rot = cr.Rotation(workloads.sylvester_rotation(256))
     x = torch.empty((0, 256), dtype=torch.bfloat16, device="cuda")
