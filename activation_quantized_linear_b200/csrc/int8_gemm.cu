@@ -68,7 +68,11 @@ struct Cfg {
   // each epilogue warp's copy of a tile's 256 bias values and 256 weight
   // scales (float)
   static constexpr int kEpiWarpBytes = 2 * BN * 4;
-  static constexpr size_t kSmem = 1024 + kStages * kStageBytes + 256 + 4 * kEpiWarpBytes;
+  // each epilogue warp's 32 x 32 tile of 16-bit outputs, staged so that the
+  // global stores write whole 64-byte row segments
+  static constexpr int kEpiStageBytes = 32 * 64;
+  static constexpr size_t kSmem =
+      1024 + kStages * kStageBytes + 256 + 4 * kEpiWarpBytes + 4 * kEpiStageBytes;
   // bytes that complete one stage on the leader's full barrier (both CTAs' loads)
   static constexpr uint32_t kTxBytes = 2 * kStageBytes;
 };
@@ -141,17 +145,15 @@ __device__ __forceinline__ float widen16(uint16_t v, bool f16) {
 // 32 outputs of one row: y = f16(float(acc) * scale [* s_w[col]] + bias[col]),
 // in bf16 or fp16 (f16), rounded once from the fp32 FMA, with the tile's bias
 // and weight scales read from the warp's shared-memory copy (float; `bias`
-// null: none, `s_w` null: per tensor).  The accumulator columns hold int32
-// (kF32Acc = false) or fp32 (true: scale is 1, so y = f16(acc + bias)).
-// `valid` (16 or 32) of the 32 columns exist.
+// null: none, `s_w` null: per tensor), as 16 words of two 16-bit values.  The
+// accumulator columns hold int32 (kF32Acc = false) or fp32 (true: scale is 1,
+// so y = f16(acc + bias)).  Columns past a half-filled chunk read staged
+// zeros and are not stored.
 template <bool kF32Acc>
-__device__ __forceinline__ void store_row32_staged(uint16_t* dst, const uint32_t (&r)[32], float scale,
-                                                   const float* s_w, const float* bias, int valid,
-                                                   bool f16) {
-  uint32_t w[16];
+__device__ __forceinline__ void row32_words(uint32_t (&w)[16], const uint32_t (&r)[32], float scale,
+                                            const float* s_w, const float* bias, bool f16) {
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
-    // columns past a half-filled chunk read staged zeros and are not stored
     const int col = 2 * i;
     float lo = kF32Acc ? __uint_as_float(r[2 * i]) : __int2float_rn(static_cast<int32_t>(r[2 * i]));
     float hi = kF32Acc ? __uint_as_float(r[2 * i + 1])
@@ -169,14 +171,13 @@ __device__ __forceinline__ void store_row32_staged(uint16_t* dst, const uint32_t
       w[i] = *reinterpret_cast<const uint32_t*>(&h);
     }
   }
-  uint4* q = reinterpret_cast<uint4*>(dst);
-  q[0] = make_uint4(w[0], w[1], w[2], w[3]);
-  q[1] = make_uint4(w[4], w[5], w[6], w[7]);
-  if (valid == 32) {
-    q[2] = make_uint4(w[8], w[9], w[10], w[11]);
-    q[3] = make_uint4(w[12], w[13], w[14], w[15]);
-  }
 }
+
+// 16-byte unit k of row r (0..31) of an epilogue warp's 32 x 32 staging tile
+// of 16-bit outputs (64-byte rows).  The unit index is XOR-ed with bits 1..2 of
+// the row: a quarter-warp writing one unit of rows r..r+7, or reading the four
+// units of two rows, then touches eight distinct 16-byte bank groups.
+__device__ __forceinline__ int stage_unit(int r, int k) { return r * 4 + (k ^ ((r >> 1) & 3)); }
 
 __device__ __forceinline__ void store_s32_row32(int32_t* dst, const uint32_t (&r)[32], int valid) {
   uint4* q = reinterpret_cast<uint4*>(dst);
@@ -371,6 +372,8 @@ __device__ __forceinline__ void gemm_pair(const CUtensorMap& tmA, const CUtensor
     // this warp's copy of the tile's factors: bias [BN], weight scales [BN]
     float* ep_bias = ep_all + (warp - 2) * (C::kEpiWarpBytes / 4);
     float* ep_sw = ep_bias + BN;
+    uint4* ep_stage = reinterpret_cast<uint4*>(ep_all + 4 * (C::kEpiWarpBytes / 4)) +
+                      (warp - 2) * (C::kEpiStageBytes / 16);
     const bool has_bias = p.bias != nullptr;
     const bool chan_sw = kKind == kKindI8 && p.per_channel_scale && !p.out_s32;
     int local = 0;
@@ -437,15 +440,38 @@ __device__ __forceinline__ void gemm_pair(const CUtensorMap& tmA, const CUtensor
         ptx::tmem_ld_32x32b_x32(t_base + c * 32, r);
         ptx::tmem_ld_wait();
         const int64_t n0 = static_cast<int64_t>(nb) * BN + c * 32;
-        const int valid = n0 + 32 <= p.N ? 32 : (n0 + 16 <= p.N ? 16 : 0);
-        if (row_ok && valid && in_bounds(m < m_limit && n0 + valid <= p.N, p.status)) {
-          if (kKind == kKindI8 && p.out_s32) {
+        const int valid = n0 + 32 <= p.N ? 32 : (n0 + 16 <= p.N ? 16 : 0);  // warp-uniform
+        if (valid == 0) continue;
+        if (kKind == kKindI8 && p.out_s32) {
+          if (row_ok && in_bounds(m < m_limit && n0 + valid <= p.N, p.status)) {
             store_s32_row32(static_cast<int32_t*>(p.out) + m * p.N + n0, r, valid);
-          } else {
-            store_row32_staged<kKind != kKindI8>(static_cast<uint16_t*>(p.out) + m * p.N + n0, r,
-                                                 scale, chan_sw ? ep_sw + c * 32 : nullptr,
-                                                 has_bias ? ep_bias + c * 32 : nullptr, valid,
-                                                 p.out_f16 != 0);
+          }
+          continue;
+        }
+        // Lane i computes row i of the warp's 32 x 32 chunk and stages it;
+        // then each store instruction writes 8 rows x 64 contiguous bytes
+        // (lane i: row 8 j + i / 4, unit i % 4), where one row per lane
+        // would touch 32 lines with 16 bytes each.
+        uint32_t w[16];
+        row32_words<kKind != kKindI8>(w, r, scale, chan_sw ? ep_sw + c * 32 : nullptr,
+                                      has_bias ? ep_bias + c * 32 : nullptr, p.out_f16 != 0);
+        __syncwarp();  // the previous chunk's staged rows are read out
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          ep_stage[stage_unit(static_cast<int>(lane), k)] =
+              make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+        }
+        __syncwarp();
+        const int unit_k = static_cast<int>(lane & 3);
+        const int64_t m_warp = m - static_cast<int64_t>(lane);  // row 0 of the warp's 32
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int rr = 8 * j + static_cast<int>(lane >> 2);
+          const int64_t mm = m_warp + rr;
+          const uint4 v = ep_stage[stage_unit(rr, unit_k)];
+          if (mm < p.M && 8 * unit_k < valid &&
+              in_bounds(mm < m_limit && n0 + valid <= p.N, p.status)) {
+            *reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + mm * p.N + n0 + 8 * unit_k) = v;
           }
         }
       }
