@@ -45,11 +45,11 @@ INT8_PER_BF16 = 2.0  # nominal dense int8 : bf16 tensor throughput (4.5 : 2.25 P
 NCU_TRAFFIC = {
     ("int8_gemm_tcgen05", "zimage_dit_block"): (120.24e6 + 102.27e6 + 151.76e6) / 3,
     ("int8_gemm_tcgen05", "wan22_a14b_video_dit"):
-        ((162.74e6 + 210.68e6) + (154.14e6 + 187.61e6) + (551.94e6 + 69.75e6)) / 3,
+        ((187.12e6 + 217.64e6) + (173.47e6 + 193.75e6) + (565.78e6 + 70.48e6)) / 3,
 }
 NCU_TRAFFIC_SOURCE_SHA = {
     ("int8_gemm_tcgen05", "zimage_dit_block"): "401d1e52793f0ba8",
-    ("int8_gemm_tcgen05", "wan22_a14b_video_dit"): "6ae71c4bca93d063",
+    ("int8_gemm_tcgen05", "wan22_a14b_video_dit"): "15eac4e6bc70d2f3",
 }
 
 
