@@ -442,6 +442,8 @@ def run_ours(args, lins):
                            f"nominal int8:bf16",
             "int8_issue_loop_tops": issue_tops,
             "frac_of_issue_loop": gemm_tops / issue_tops if issue_tops else None,
+            # context: the cuBLAS reference looped for seconds under the power cap
+            "frac_of_sustained": gemm_tops / (bf16_sust * INT8_PER_BF16),
         },
         "kernels": {
             "rotate_quant_act": {"ms": rqa_mean.tolist(), "GB/s": rqa_gbs,
