@@ -287,18 +287,10 @@ __device__ __forceinline__ uint32_t pack4(uint32_t a, uint32_t b, uint32_t c, ui
 }
 
 // Writes the low byte of each half of R (a code in two's complement) where
-// fwht32 left that element; `base` = first element of the lane's chunk, and
-// only lanes with `store` write.  Every lane of the warp calls it.  At
-// G = 256 lane (g, t) holds word s (4 codes) of its group at byte 32 s + 4 t;
-// the warp's four groups go through its exchange slot `stage` (free after
-// fwht32; groups 288 bytes apart, so the word stores hit 32 distinct banks)
-// and come back as the lane's own 32 contiguous codes, two 16-byte stores
-// that each cover whole 32-byte sectors (lanes t >= 4 read their halves in
-// the other order: each 8-lane phase then reads 8 distinct 16-byte bank
-// groups).
+// fwht32 left that element; `base` = first element of the lane's chunk.
 template <int G>
 __device__ __forceinline__ void store_code_bytes(int8_t* base, const uint64_t (&R)[kPairs],
-                                                 uint32_t lane, uint32_t stage, bool store) {
+                                                 uint32_t lane) {
   uint32_t w[8];
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
@@ -309,24 +301,10 @@ __device__ __forceinline__ void store_code_bytes(int8_t* base, const uint64_t (&
   }
   if constexpr (G == 256) {
     const uint32_t t = lane & 7;
-    const uint32_t gs = stage + 288 * (lane >> 3);
+    int8_t* grp = base - kVec * t;
 #pragma unroll
-    for (int s = 0; s < 8; ++s) {
-      asm volatile("st.shared.b32 [%0], %1;" ::"r"(gs + 32 * s + 4 * t), "r"(w[s]) : "memory");
-    }
-    __syncwarp();
-    const uint32_t h0 = t >> 2;
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const uint32_t half = h0 ^ static_cast<uint32_t>(h);
-      uint4 v;
-      asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                   : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                   : "r"(gs + 32 * t + 16 * half)
-                   : "memory");
-      if (store) *reinterpret_cast<uint4*>(base + 16 * half) = v;
-    }
-  } else if (store) {
+    for (int s = 0; s < 8; ++s) *reinterpret_cast<uint32_t*>(grp + 32 * s + 4 * t) = w[s];
+  } else {
     uint4* q = reinterpret_cast<uint4*>(base);
     q[0] = make_uint4(w[0], w[1], w[2], w[3]);
     q[1] = make_uint4(w[4], w[5], w[6], w[7]);
@@ -337,19 +315,18 @@ __device__ __forceinline__ void store_code_bytes(int8_t* base, const uint64_t (&
 // against 1.5 * 2^23 leaves each code in the low byte of its float.
 template <int G>
 __device__ __forceinline__ void store_codes32(int8_t* base, const uint64_t (&P)[kPairs], float mul,
-                                             uint32_t lane, uint32_t stage, bool store) {
+                                             uint32_t lane) {
   const uint64_t m2 = pk(mul, mul), magic2 = pk(kRoundMagic, kRoundMagic);
   uint64_t R[kPairs];
 #pragma unroll
   for (int i = 0; i < kPairs; ++i) R[i] = fma2(P[i], m2, magic2);
-  store_code_bytes<G>(base, R, lane, stage, store);
+  store_code_bytes<G>(base, R, lane);
 }
 
 // Exact-division codes rne(v * norm / s), for scales so small that 1/s overflows.
 template <int G>
 __device__ __forceinline__ void store_codes32_div(int8_t* base, const uint64_t (&P)[kPairs],
-                                                  float norm, float s, uint32_t lane, uint32_t stage,
-                                                  bool store) {
+                                                  float norm, float s, uint32_t lane) {
   uint64_t R[kPairs];
 #pragma unroll
   for (int i = 0; i < kPairs; ++i) {
@@ -357,7 +334,7 @@ __device__ __forceinline__ void store_codes32_div(int8_t* base, const uint64_t (
     const float b = fminf(fmaxf(rintf(__fdiv_rn(phi(P[i]) * norm, s)), -127.f), 127.f);
     R[i] = pk(a + kRoundMagic, b + kRoundMagic);
   }
-  store_code_bytes<G>(base, R, lane, stage, store);
+  store_code_bytes<G>(base, R, lane);
 }
 
 // The exact products s * v of a pair, each rounded once to nearest-even into a
@@ -606,10 +583,10 @@ __global__ void __launch_bounds__(kMaxThreads, kMinBlocks) rotate_quant_act_hada
       team_barrier<kTeams>(team, bar_threads);
       amax = warp_max(static_cast<int>(lane) < team_warps ? rb_red[team * team_warps + lane] : 0.f);
     }
-    if (row >= M) continue;  // the team's row is past the end (uniform over the team)
+    if (!ok) continue;
     // debug build: the token's codes and scale must lie inside xq and s_tok
     const int64_t row_limit = CONVROT_DEBUG && fault == kFaultShortRows ? M - 1 : M;
-    const bool store = t < nch && in_bounds(row < row_limit && (t + 1) * kVec <= K, status);
+    if (!in_bounds(row < row_limit && (t + 1) * kVec <= K, status)) continue;
     // s_tok = max |x_rot| / 127, correctly rounded without a division.  With
     // a = amax * norm (exact) and m any float32 rounding midpoint of a / 127,
     // a - 127 m is an odd multiple of half the quotient's ulp (a's bits are
@@ -618,13 +595,13 @@ __global__ void __launch_bounds__(kMaxThreads, kMinBlocks) rotate_quant_act_hada
     // the quotient is subnormal.  The float64 product a * RN(1/127) is within
     // 2^-52 (relative) of a / 127, so its one rounding to float32 is RN(a / 127).
     const float sc = static_cast<float>(static_cast<double>(amax * norm) * (1.0 / 127.0));
-    if (t == 0 && store) s_tok[row] = sc;
+    if (t == 0) s_tok[row] = sc;
     const float mul = norm * (sc > 0.f ? 1.f / sc : 0.f);  // exact scaling: norm is a power of two
     int8_t* dst = xq + row * K + static_cast<int64_t>(t) * kVec;
-    if (mul <= 3.0e38f) {  // uniform over the team
-      store_codes32<G>(dst, P, mul, lane, xch, store);
+    if (mul <= 3.0e38f) {
+      store_codes32<G>(dst, P, mul, lane);
     } else {
-      store_codes32_div<G>(dst, P, norm, sc, lane, xch, store);
+      store_codes32_div<G>(dst, P, norm, sc, lane);
     }
   }
 }
@@ -715,12 +692,13 @@ __global__ void __launch_bounds__(256, MODE == kFlatDequant ? 3 : 4) hadamard_fl
     if constexpr (MODE == kFlatAbsmax) {
       if (ok) run_max = fmaxf(run_max, absmax32(P));
     } else if constexpr (MODE == kFlatQuant) {
-      const bool store = ok && in_bounds((G == 256 ? (c | 7) : c) < chunk_limit, status);
-      int8_t* dst = static_cast<int8_t*>(out) + c * kVec;
-      if (mul <= 3.0e38f) {  // uniform over the grid
-        store_codes32<G>(dst, P, mul, lane, aux, store);
-      } else {
-        store_codes32_div<G>(dst, P, norm, s, lane, aux, store);
+      if (ok && in_bounds((G == 256 ? (c | 7) : c) < chunk_limit, status)) {
+        int8_t* dst = static_cast<int8_t*>(out) + c * kVec;
+        if (mul <= 3.0e38f) {
+          store_codes32<G>(dst, P, mul, lane);
+        } else {
+          store_codes32_div<G>(dst, P, norm, s, lane);
+        }
       }
     } else {
       // output row of chunk c: c / (K / 32) as a multiply and shift (row_reciprocal)
