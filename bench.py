@@ -43,12 +43,12 @@ INT8_PER_BF16 = 2.0  # nominal dense int8 : bf16 tensor throughput (4.5 : 2.25 P
 # averaged over the GEMM launches of one step of a workload, valid only for the
 # kernel source they were taken on (first 16 hex digits of its sha256).
 NCU_TRAFFIC = {
-    ("int8_gemm_tcgen05", "zimage_dit_block"): (120.24e6 + 102.27e6 + 151.76e6) / 3,
+    ("int8_gemm_tcgen05", "zimage_dit_block"): ((62.16e6 + 69.42e6) + (57.17e6 + 54.22e6) + (143.70e6 + 21.10e6)) / 3,
     ("int8_gemm_tcgen05", "wan22_a14b_video_dit"):
         ((187.12e6 + 217.64e6) + (173.47e6 + 193.75e6) + (565.78e6 + 70.48e6)) / 3,
 }
 NCU_TRAFFIC_SOURCE_SHA = {
-    ("int8_gemm_tcgen05", "zimage_dit_block"): "401d1e52793f0ba8",
+    ("int8_gemm_tcgen05", "zimage_dit_block"): "15eac4e6bc70d2f3",
     ("int8_gemm_tcgen05", "wan22_a14b_video_dit"): "15eac4e6bc70d2f3",
 }
 
