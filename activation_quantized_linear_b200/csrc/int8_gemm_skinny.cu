@@ -429,6 +429,7 @@ cudaError_t launch_nt(const GemmArgs& a, SkinnyParams p, cudaStream_t stream) {
 }  // namespace
 
 cudaError_t launch_int8_gemm_skinny(const GemmArgs& a, cudaStream_t stream) {
+  if (int8_gemv_applies(a)) return launch_int8_gemv(a, stream);
   SkinnyParams p;
   cudaError_t e = status_word(&p.status);
   if (e != cudaSuccess) return e;

@@ -98,8 +98,19 @@ struct GemmArgs {
 // cudaErrorInvalidValue if a tensor map cannot be encoded.
 cudaError_t launch_int8_gemm(const GemmArgs& a, cudaStream_t stream);
 
-// The few-token variant (M <= 128): swap-AB with the K split over a cluster.
+// The few-token variant (M <= 128): swap-AB with the K split over a cluster;
+// up to kGemvMaxTokens tokens it hands over to the dp4a product below.
 cudaError_t launch_int8_gemm_skinny(const GemmArgs& a, cudaStream_t stream);
+
+// One or two tokens, whose codes (rounded up to 1 or 2 token rows of K bytes)
+// fit kGemvMaxCodeBytes of shared memory: warps streaming whole weight rows
+// with dp4a (int8_gemv.cu).  Same results as the tensor-core GEMMs.  (At 4
+// and 8 tokens the per-token dot products made it slower than the swap-AB
+// kernel on every measured weight.)
+constexpr int kGemvMaxTokens = 2;
+constexpr int64_t kGemvMaxCodeBytes = 64 << 10;
+bool int8_gemv_applies(const GemmArgs& a);
+cudaError_t launch_int8_gemv(const GemmArgs& a, cudaStream_t stream);
 
 // y = f16(x W^T + bias) with 16-bit operands (a.ops16, a.A16, a.B16; bf16 or
 // fp16 as a.out_f16), fp32 accumulation on the same CTA-pair pipeline.

@@ -98,7 +98,7 @@ def _untouched(t):
     return bool((t.reshape(-1).view(torch.uint8) == SENTINEL).all())
 
 
-@pytest.mark.parametrize("M", [300, 16])
+@pytest.mark.parametrize("M", [300, 16, 2])
 def test_debug_library_matches_release_bit_for_bit(libs, M):
     cr, dbg = libs
     L = DebugLayer(cr, dbg, M, 512, 1024, seed=M)
@@ -117,7 +117,7 @@ def test_debug_library_matches_release_bit_for_bit(libs, M):
     L.close()
 
 
-@pytest.mark.parametrize("M", [300, 16])
+@pytest.mark.parametrize("M", [300, 16, 2])
 def test_short_rows_fault_is_caught_and_skipped(libs, M):
     """The kernels believe the outputs one row shorter: the last row's stores
     are out of range, caught, skipped and reported; nothing else changes."""

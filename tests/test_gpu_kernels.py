@@ -57,6 +57,11 @@ def _codes(rng, shape):
 GEMM_SHAPES = [
     (1, 16, 16), (7, 144, 64), (128, 256, 128), (129, 272, 144), (257, 512, 1024),
     (300, 1024, 3840), (64, 1024, 1024), (1000, 528, 2048), (33, 4096, 256), (97, 1008, 4096),
+    # one or two tokens whose codes fit 64 KB take the dp4a product: one, two
+    # and eight 4 KB row blocks, several rows per warp, the largest K it takes
+    # and the first past it (swap-AB); and a few more swap-AB token counts
+    (2, 21504, 3072), (1, 1040, 8192), (2, 528, 32768), (2, 528, 32784), (1, 4096, 4096),
+    (5, 1040, 8192), (8, 528, 8192), (3, 4096, 4096),
 ]
 
 
@@ -72,11 +77,13 @@ def test_int8_gemm_s32_bit_exact(M, N, K):
     np.testing.assert_array_equal(acc.cpu().numpy(), oracle.int8_gemm_acc(a, b))
 
 
-@pytest.mark.parametrize("M,N,K", [(130, 272, 15360), (130, 144, 131072), (3, 144, 131072)])
+@pytest.mark.parametrize("M,N,K", [(130, 272, 15360), (130, 144, 131072), (3, 144, 131072),
+                                   (2, 144, 16384)])
 def test_int8_gemm_s32_extremes(M, N, K):
     """Largest accumulators: |acc| = 127^2 K, at the workloads' K = 15360 and at
-    the interface's limit K = 131072 (127^2 * 131072 < 2^31), on both GEMM
-    paths (CTA pairs for M > 128, swap-AB below)."""
+    the interface's limit K = 131072 (127^2 * 131072 < 2^31), on the three
+    GEMM paths (CTA pairs for M > 128, swap-AB below, the dp4a product for one
+    or two tokens with at most 64 KB of codes: M = 2, K = 16384)."""
     a = np.full((M, K), 127, np.int8)
     a[1::2] = -127
     a[min(5, M - 1), ::2] = 0
@@ -119,6 +126,8 @@ def _assert_epilogue_close(y_gpu, acc, s_tok, s_w, bias):
 @pytest.mark.parametrize("M,N,K,with_bias,per_channel", [
     (64, 1024, 1024, True, False), (129, 272, 144, False, False), (7, 144, 64, True, True),
     (257, 512, 256, True, True), (100, 1008, 2048, True, True),
+    (3, 1040, 4096, True, False), (1, 2048, 3072, False, True), (8, 528, 8192, True, True),
+    (2, 1040, 4096, True, True),
 ])
 def test_int8_gemm_epilogue(M, N, K, with_bias, per_channel):
     rng = np.random.default_rng(M + N + K)
