@@ -553,7 +553,7 @@ def run_sweep(args):
     sw1 = torch.tensor([1e-3], device="cuda")
     for Kc, Nc, copies in ((4096, 4096, 8), (3072, 21504, 3), (3840, 11520, 4), (10240, 3840, 4)):
         Ws = [torch.randint(-127, 128, (Nc, Kc), dtype=torch.int8, device="cuda") for _ in range(copies)]
-        for Mc in (1, 16, 64, 128):
+        for Mc in (1, 2, 16, 64, 128):  # 1-2 tokens: the dp4a product; more: swap-AB
             xq = torch.randint(-127, 128, (Mc, Kc), dtype=torch.int8, device="cuda")
             st = torch.rand(Mc, device="cuda") * 1e-3
             y = torch.empty((Mc, Nc), dtype=torch.bfloat16, device="cuda")
