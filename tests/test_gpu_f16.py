@@ -137,7 +137,7 @@ def test_dequant_derotate_f16_scales(G):
 
 @pytest.mark.parametrize("M,N,K,with_bias,per_channel", [
     (300, 1024, 1024, True, False), (129, 272, 144, False, True), (7, 144, 64, True, False),
-    (64, 512, 512, True, True),
+    (64, 512, 512, True, True), (2, 528, 2048, True, True),  # two tokens: the dp4a product
 ])
 def test_int8_gemm_f16(M, N, K, with_bias, per_channel):
     rng = np.random.default_rng(M * N + K)
