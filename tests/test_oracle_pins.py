@@ -370,8 +370,23 @@ def check_per_channel_properties(o):
             raise AssertionError("a weight scale of the wrong length was accepted")
 
 
+def check_bit_patterns(o):
+    """16-bit encodings written out from the formats' definitions: IEEE 754
+    binary16 (1 sign, 5 exponent bits biased by 15, 10 fraction bits) and
+    bfloat16 (the upper half of binary32: 8 exponent bits biased by 127, 7
+    fraction bits), normal and subnormal, both signs."""
+    f16 = {1.0: 0x3C00, -2.0: 0xC000, 0.5: 0x3800, 65504.0: 0x7BFF, 2.0 ** -14: 0x0400,
+           2.0 ** -24: 0x0001, 1365.0 / 4096: 0x3555, -0.0: 0x8000, -(2.0 ** -15): 0x8200}
+    bf16 = {1.0: 0x3F80, -2.0: 0xC000, 0.5: 0x3F00, 0.15625: 0x3E20, 2.0 ** -126: 0x0080,
+            2.0 ** -133: 0x0001, (2 - 2.0 ** -7) * 2.0 ** 127: 0x7F7F, -0.0: 0x8000,
+            -3.0: 0xC040}
+    for table, fn in ((f16, o.f16_bits), (bf16, o.bf16_bits)):
+        vals = np.array(list(table.keys()), np.float64)
+        np.testing.assert_array_equal(fn(vals).astype(np.int64), np.array(list(table.values())))
+
+
 CHECKS = [
-    check_per_channel_worked_example, check_per_channel_square_decode, check_per_channel_properties,
+    check_bit_patterns, check_per_channel_worked_example, check_per_channel_square_decode, check_per_channel_properties,
     check_f16_round, check_worked_example, check_block_rotate_bruteforce, check_block_rotate_direction,
     check_rotation_identity, check_round_trip, check_bf16_round, check_quantize_symmetric,
     check_act_quant_properties, check_zero_token, check_gemm_bruteforce, check_gemm_extremes,
@@ -565,7 +580,18 @@ def _bug_per_channel_codes_with_tensor_scale(W, R, per_channel=False):
     return Wq, (np.max(np.abs(W_rot), axis=1) / 127).astype(np.float32)
 
 
+def _bug_bf16_bits_low_half(v):
+    f = np.asarray(v, dtype=np.float64).astype(np.float32)
+    return (f.view(np.uint32) & 0xFFFF).astype(np.uint16)
+
+
+def _bug_f16_bits_byteswapped(v):
+    return np.asarray(v, dtype=np.float64).astype(np.float16).view(np.uint16).byteswap()
+
+
 MUTANTS = {
+    "bf16_bits_low_half": dict(bf16_bits=_bug_bf16_bits_low_half),
+    "f16_bits_byteswapped": dict(f16_bits=_bug_f16_bits_byteswapped),
     "decode_scale_on_input_axis": dict(dequant_derotate=_bug_decode_scale_on_input_axis),
     "epilogue_scale_on_token_axis": dict(epilogue=_bug_epilogue_scale_on_token_axis),
     "channel_scales_collapsed": dict(weight_scale_column=_bug_channel_scales_collapsed),
